@@ -1,0 +1,332 @@
+// C ABI of the RainFusion2.0 block-sparse attention library (include/rf2.h).
+//
+// Host code: argument validation, closed-form sizes, TMA tensor maps and
+// kernel launches.  All kernels live in this one translation unit so they
+// share the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "rf2.h"
+#include "attn.cuh"
+#include "geometry.cuh"
+#include "mask.cuh"
+#include "permute.cuh"
+#include "ptx.cuh"
+
+namespace rf2 {
+
+// Device status word: kernels OR error bits into it; rf2_device_status
+// reads and clears it.
+__device__ int g_status_word;
+
+constexpr int32_t kMaxBlocks = 4096;     // T_b limit (N <= 262,144 tokens)
+
+struct Checked {
+    int status;
+    PermGeo pg;
+    int64_t BH;
+    int32_t N, Tb, D;
+};
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static Checked check_geometry(const rf2_geometry* g)
+{
+    Checked c;
+    memset(&c, 0, sizeof c);
+    c.status = RF2_ERR_INVALID_ARGUMENT;
+    if (!g) return c;
+    if (g->batch <= 0 || g->heads <= 0 || g->frames <= 0 || g->height <= 0 || g->width <= 0 ||
+        g->win_t <= 0 || g->win_h <= 0 || g->win_w <= 0 || g->head_dim <= 0 || g->block <= 0 ||
+        (g->first_frame_sink != 0 && g->first_frame_sink != 1))
+        return c;
+    const int64_t N = (int64_t)g->frames * g->height * g->width;
+    if (N > INT32_MAX) return c;
+    c.status = RF2_ERR_UNSUPPORTED;
+    if (g->head_dim != 64 && g->head_dim != 128) return c;
+    if (g->block != kBlock) return c;
+    const int64_t Tb = (N + kBlock - 1) / kBlock;
+    if (Tb > kMaxBlocks) return c;
+    c.BH = (int64_t)g->batch * g->heads;
+    if (c.BH > (int64_t)INT32_MAX / 2) return c;
+    c.N = (int32_t)N;
+    c.Tb = (int32_t)Tb;
+    c.D = g->head_dim;
+    c.pg = make_perm_geo(g->frames, g->height, g->width, g->win_t, g->win_h, g->win_w, g->first_frame_sink);
+    c.status = RF2_OK;
+    return c;
+}
+
+static int keep_count(double keep, int32_t Tb, int32_t* n)
+{
+    if (!(keep > 0.0) || !(keep <= 1.0)) return RF2_ERR_INVALID_ARGUMENT;
+    int64_t k = (int64_t)ceil(keep * (double)Tb - 1e-9);
+    if (k < 1) k = 1;
+    if (k > Tb) k = Tb;
+    *n = (int32_t)k;
+    return RF2_OK;
+}
+
+static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg, rf2_sizes* out)
+{
+    c = check_geometry(g);
+    if (c.status != RF2_OK) return c.status;
+    int32_t n = 0;
+    const int st = keep_count(keep, c.Tb, &n);
+    if (st != RF2_OK) return st;
+    mg = make_mask_geo(c.N, n, g->first_frame_sink, g->frames, g->height * g->width);
+    const int64_t total = c.BH * mg.head_total;
+    if (total > INT32_MAX) return RF2_ERR_UNSUPPORTED;
+    if (out) {
+        out->num_tokens = c.N;
+        out->num_blocks = c.Tb;
+        out->n_keep = n;
+        out->sink_first = (mg.sink_first < c.Tb) ? mg.sink_first : -1;
+        out->row_capacity = mg.cap;
+        out->num_rows = c.BH * c.Tb;
+        out->col_idx_capacity = total;
+        out->mask_workspace_bytes = (size_t)2 * c.BH * c.Tb * c.D * sizeof(float);
+    }
+    return RF2_OK;
+}
+
+static int launch_status()
+{
+    const cudaError_t e = cudaPeekAtLastError();
+    return e == cudaSuccess ? RF2_OK : RF2_ERR_CUDA;
+}
+
+static int grid_for_rows(int64_t rows)
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t warps = (rows + 31) / 32;
+    int64_t blocks = (warps + 7) / 8;
+    const int64_t cap = (int64_t)sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return (int)blocks;
+}
+
+static int permute_impl(const rf2_geometry* geom, const void* in, void* out, void* stream, bool forward)
+{
+    Checked c = check_geometry(geom);
+    if (c.status != RF2_OK) return c.status;
+    if (!in || !out || !aligned16(in) || !aligned16(out) || in == out) return RF2_ERR_INVALID_ARGUMENT;
+    const int64_t rows = c.BH * c.N;
+    const int grid = grid_for_rows(rows);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const uint4* i4 = reinterpret_cast<const uint4*>(in);
+    uint4* o4 = reinterpret_cast<uint4*>(out);
+    if (c.D == 128) {
+        if (forward) permute_rows_kernel<128, true><<<grid, 256, 0, s>>>(i4, o4, c.pg, rows);
+        else         permute_rows_kernel<128, false><<<grid, 256, 0, s>>>(i4, o4, c.pg, rows);
+    } else {
+        if (forward) permute_rows_kernel<64, true><<<grid, 256, 0, s>>>(i4, o4, c.pg, rows);
+        else         permute_rows_kernel<64, false><<<grid, 256, 0, s>>>(i4, o4, c.pg, rows);
+    }
+    return launch_status();
+}
+
+// ---------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [BH, N, D] bf16 viewed as a 3D tensor (D, N, BH); box = 64 columns x rows,
+// 128-byte swizzle (the canonical K-major / MN-major SW128 tcgen05 layouts).
+static bool make_map(CUtensorMap* m, const void* ptr, int32_t D, int32_t N, int64_t BH, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+    const cuuint32_t box[3] = {64, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int* status_word_ptr()
+{
+    int* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_status_word) != cudaSuccess) return nullptr;
+    return p;
+}
+
+template <int D>
+static int launch_attn(const Checked& c, const MaskGeo& mg, const void* qp, const void* kp, const void* vp,
+                       const int32_t* row_start, const int32_t* row_count, const int32_t* col_idx, void* op,
+                       float* lse, cudaStream_t s)
+{
+    using Cfg = AttnCfg<D>;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, qp, D, c.N, c.BH, 128) || !make_map(&mk, kp, D, c.N, c.BH, 64) ||
+        !make_map(&mv, vp, D, c.N, c.BH, 64))
+        return RF2_ERR_CUDA;
+    int* status = status_word_ptr();
+    if (!status) return RF2_ERR_CUDA;
+    AttnArgs a;
+    a.row_start = row_start;
+    a.row_count = row_count;
+    a.col_idx = col_idx;
+    a.op = reinterpret_cast<uint16_t*>(op);
+    a.lse = lse;
+    a.status = status;
+    a.N = c.N;
+    a.Tb = c.Tb;
+    a.pairs = (c.Tb + 1) / 2;
+    a.sink_pairs = (mg.sink_first < c.Tb) ? a.pairs - mg.sink_first / 2 : 0;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    const size_t smem = Cfg::smem_bytes(c.Tb);
+    if (cudaFuncSetAttribute(block_sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return RF2_ERR_CUDA;
+    const int64_t grid = c.BH * a.pairs;
+    block_sparse_attn_kernel<D><<<(unsigned)grid, Cfg::THREADS, smem, s>>>(mq, mk, mv, a);
+    return launch_status();
+}
+
+template <int D, int R>
+static int launch_select(const Checked& c, const MaskGeo& mg, const float* means, int32_t* row_start,
+                         int32_t* row_count, int32_t* col_idx, cudaStream_t s)
+{
+    const size_t smem = SelectSmem<D, R>::bytes(c.Tb);
+    if (cudaFuncSetAttribute(select_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return RF2_ERR_CUDA;
+    dim3 grid((c.Tb + R - 1) / R, (unsigned)c.BH);
+    select_kernel<D, R><<<grid, kSelThreads, smem, s>>>(means, row_start, row_count, col_idx, mg, c.BH,
+                                                       (float)(1.0 / sqrt((double)D)));
+    return launch_status();
+}
+
+}  // namespace rf2
+
+using namespace rf2;
+
+extern "C" {
+
+const char* rf2_status_string(int status)
+{
+    switch (status) {
+    case RF2_OK: return "ok";
+    case RF2_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case RF2_ERR_UNSUPPORTED: return "unsupported geometry";
+    case RF2_ERR_INSUFFICIENT_WORKSPACE: return "workspace too small";
+    case RF2_ERR_CUDA: return "CUDA error";
+    case RF2_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+    }
+}
+
+int rf2_query(const rf2_geometry* geom, double keep_ratio, rf2_sizes* out)
+{
+    if (!out) return RF2_ERR_INVALID_ARGUMENT;
+    Checked c;
+    MaskGeo mg;
+    return sizes_for(geom, keep_ratio, c, mg, out);
+}
+
+int rf2_permutation_index(const rf2_geometry* geom, int32_t* perm)
+{
+    Checked c = check_geometry(geom);
+    if (c.status != RF2_OK) return c.status;
+    if (!perm) return RF2_ERR_INVALID_ARGUMENT;
+    for (int32_t p = 0; p < c.N; ++p) perm[p] = perm_src(c.pg, p);
+    return RF2_OK;
+}
+
+int rf2_permute(const rf2_geometry* geom, const void* x, void* xp, void* stream)
+{
+    return permute_impl(geom, x, xp, stream, true);
+}
+
+int rf2_unpermute(const rf2_geometry* geom, const void* xp, void* x, void* stream)
+{
+    return permute_impl(geom, xp, x, stream, false);
+}
+
+int rf2_predict_mask(const rf2_geometry* geom, const void* qp, const void* kp, double keep_ratio,
+                     int32_t* row_start, int32_t* row_count, int32_t* col_idx, void* workspace,
+                     size_t workspace_bytes, void* stream)
+{
+    Checked c;
+    MaskGeo mg;
+    rf2_sizes sz;
+    const int st = sizes_for(geom, keep_ratio, c, mg, &sz);
+    if (st != RF2_OK) return st;
+    if (!qp || !kp || !row_start || !row_count || !col_idx || !workspace) return RF2_ERR_INVALID_ARGUMENT;
+    if (!aligned16(qp) || !aligned16(kp) || !aligned16(workspace) || !aligned16(row_start) ||
+        !aligned16(row_count) || !aligned16(col_idx))
+        return RF2_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < sz.mask_workspace_bytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* means = reinterpret_cast<float*>(workspace);
+    const int64_t warps = 2 * c.BH * c.Tb;
+    const unsigned grid = (unsigned)((warps + 7) / 8);
+    if (c.D == 128)
+        block_mean_kernel<128><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
+                                                     reinterpret_cast<const uint4*>(kp), means, c.N, c.Tb, c.BH);
+    else
+        block_mean_kernel<64><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
+                                                    reinterpret_cast<const uint4*>(kp), means, c.N, c.Tb, c.BH);
+    int r = launch_status();
+    if (r != RF2_OK) return r;
+    if (c.Tb <= 2048)
+        r = (c.D == 128) ? launch_select<128, 16>(c, mg, means, row_start, row_count, col_idx, s)
+                         : launch_select<64, 16>(c, mg, means, row_start, row_count, col_idx, s);
+    else
+        r = (c.D == 128) ? launch_select<128, 8>(c, mg, means, row_start, row_count, col_idx, s)
+                         : launch_select<64, 8>(c, mg, means, row_start, row_count, col_idx, s);
+    return r;
+}
+
+int rf2_block_sparse_attn(const rf2_geometry* geom, const void* qp, const void* kp, const void* vp,
+                          const int32_t* row_start, const int32_t* row_count, const int32_t* col_idx,
+                          void* op, float* lse, void* stream)
+{
+    const Checked c = check_geometry(geom);
+    if (c.status != RF2_OK) return c.status;
+    const MaskGeo mg = make_mask_geo(c.N, 1, geom->first_frame_sink, geom->frames, geom->height * geom->width);
+    if (!qp || !kp || !vp || !row_start || !row_count || !col_idx || !op) return RF2_ERR_INVALID_ARGUMENT;
+    if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(op) || !aligned16(row_start) ||
+        !aligned16(row_count) || !aligned16(col_idx) || (lse && !aligned16(lse)))
+        return RF2_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return (c.D == 128) ? launch_attn<128>(c, mg, qp, kp, vp, row_start, row_count, col_idx, op, lse, s)
+                        : launch_attn<64>(c, mg, qp, kp, vp, row_start, row_count, col_idx, op, lse, s);
+}
+
+int rf2_device_status(void* stream)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return RF2_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof v) != cudaSuccess) return RF2_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero) != cudaSuccess) return RF2_ERR_CUDA;
+    return (v & kDevErrTimeout) ? RF2_ERR_TIMEOUT : RF2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,226 @@
+"""Python binding of the C ABI in ``include/rf2.h`` (ctypes; marshalling only).
+
+Every step of the path runs in ``librf2.so``'s CUDA kernels.  PyTorch only
+provides device memory and the current stream.  There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librf2.so")
+
+RF2_OK = 0
+RF2_ERR_INVALID_ARGUMENT = 1
+RF2_ERR_UNSUPPORTED = 2
+RF2_ERR_INSUFFICIENT_WORKSPACE = 3
+RF2_ERR_CUDA = 4
+RF2_ERR_TIMEOUT = 5
+
+# Every entry point declared in include/rf2.h.
+EXPORTED = (
+    "rf2_status_string", "rf2_query", "rf2_permutation_index", "rf2_permute", "rf2_unpermute",
+    "rf2_predict_mask", "rf2_block_sparse_attn", "rf2_device_status",
+)
+
+
+class Geometry(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "heads", "head_dim", "frames", "height", "width",
+        "win_t", "win_h", "win_w", "block", "first_frame_sink")]
+
+
+class Sizes(ctypes.Structure):
+    _fields_ = [
+        ("num_tokens", ctypes.c_int64),
+        ("num_blocks", ctypes.c_int32),
+        ("n_keep", ctypes.c_int32),
+        ("sink_first", ctypes.c_int32),
+        ("row_capacity", ctypes.c_int32),
+        ("num_rows", ctypes.c_int64),
+        ("col_idx_capacity", ctypes.c_int64),
+        ("mask_workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class Rf2Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """Load librf2.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} (run image_dits_b200.build.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, f64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
+        G = ctypes.POINTER(Geometry)
+        L.rf2_status_string.argtypes = [i32]
+        L.rf2_status_string.restype = ctypes.c_char_p
+        L.rf2_query.argtypes = [G, f64, ctypes.POINTER(Sizes)]
+        L.rf2_permutation_index.argtypes = [G, vp]
+        L.rf2_permute.argtypes = [G, vp, vp, vp]
+        L.rf2_unpermute.argtypes = [G, vp, vp, vp]
+        L.rf2_predict_mask.argtypes = [G, vp, vp, f64, vp, vp, vp, vp, sz, vp]
+        L.rf2_block_sparse_attn.argtypes = [G, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.rf2_device_status.argtypes = [vp]
+        for name in EXPORTED:
+            if name != "rf2_status_string":
+                getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().rf2_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != RF2_OK:
+        raise Rf2Error(status, what)
+
+
+def make_geometry(batch, heads, head_dim, frames, height, width, win_t, win_h, win_w, sink, block=64) -> Geometry:
+    return Geometry(batch, heads, head_dim, frames, height, width, win_t, win_h, win_w, block, int(bool(sink)))
+
+
+def geometry_of(wl, batch: int | None = None) -> Geometry:
+    """Geometry of a ``workload.Workload``."""
+    return make_geometry(wl.batch if batch is None else batch, wl.heads, wl.head_dim, wl.frames, wl.height,
+                         wl.width, wl.win_t, wl.win_h, wl.win_w, wl.sink)
+
+
+def query(geom: Geometry, keep: float = 1.0) -> Sizes:
+    out = Sizes()
+    _check(lib().rf2_query(ctypes.byref(geom), float(keep), ctypes.byref(out)), "rf2_query")
+    return out
+
+
+def permutation_index(geom: Geometry) -> np.ndarray:
+    n = geom.frames * geom.height * geom.width
+    perm = np.empty(n, dtype=np.int32)
+    _check(lib().rf2_permutation_index(ctypes.byref(geom), perm.ctypes.data), "rf2_permutation_index")
+    return perm
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_qkv(geom: Geometry, *ts):
+    shape = (geom.batch, geom.heads, geom.frames * geom.height * geom.width, geom.head_dim)
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and tuple(t.shape) == shape):
+            raise ValueError(f"expected a contiguous CUDA bf16 tensor of shape {shape}, got "
+                             f"{tuple(t.shape)} {t.dtype} {t.device}")
+
+
+def permute(geom: Geometry, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _check_qkv(geom, x)
+    out = torch.empty_like(x) if out is None else out
+    _check_qkv(geom, out)
+    _check(lib().rf2_permute(ctypes.byref(geom), x.data_ptr(), out.data_ptr(), _stream(stream)), "rf2_permute")
+    return out
+
+
+def unpermute(geom: Geometry, xp: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _check_qkv(geom, xp)
+    out = torch.empty_like(xp) if out is None else out
+    _check_qkv(geom, out)
+    _check(lib().rf2_unpermute(ctypes.byref(geom), xp.data_ptr(), out.data_ptr(), _stream(stream)), "rf2_unpermute")
+    return out
+
+
+@dataclass
+class BlockMask:
+    """CSR block mask: row r = (b*heads + h)*T_b + i keeps
+    col_idx[row_start[r] : row_start[r] + row_count[r]] (ascending)."""
+    row_start: torch.Tensor
+    row_count: torch.Tensor
+    col_idx: torch.Tensor
+    sizes: Sizes
+
+    def dense(self) -> np.ndarray:
+        """[B*H, T_b, T_b] uint8 on the host (for tests)."""
+        Tb = self.sizes.num_blocks
+        rs = self.row_start.cpu().numpy().astype(np.int64)
+        rc = self.row_count.cpu().numpy().astype(np.int64)
+        ci = self.col_idx.cpu().numpy()
+        out = np.zeros((rs.size, Tb), np.uint8)
+        for r in range(rs.size):
+            out[r, ci[rs[r]:rs[r] + rc[r]]] = 1
+        return out.reshape(-1, Tb, Tb)
+
+    def kept_pairs(self) -> int:
+        return int(self.row_count.sum().item())
+
+
+def alloc_mask(geom: Geometry, keep: float, device) -> tuple:
+    sz = query(geom, keep)
+    row_start = torch.empty(sz.num_rows, dtype=torch.int32, device=device)
+    row_count = torch.empty(sz.num_rows, dtype=torch.int32, device=device)
+    col_idx = torch.empty(max(1, sz.col_idx_capacity), dtype=torch.int32, device=device)
+    ws = torch.empty(max(16, sz.mask_workspace_bytes), dtype=torch.uint8, device=device)
+    return BlockMask(row_start, row_count, col_idx, sz), ws
+
+
+def predict_mask(geom: Geometry, qp: torch.Tensor, kp: torch.Tensor, keep: float, mask: BlockMask | None = None,
+                 workspace: torch.Tensor | None = None, stream=None) -> BlockMask:
+    _check_qkv(geom, qp, kp)
+    if mask is None or workspace is None:
+        m2, ws2 = alloc_mask(geom, keep, qp.device)
+        mask = mask or m2
+        workspace = ws2 if workspace is None else workspace
+    _check(lib().rf2_predict_mask(ctypes.byref(geom), qp.data_ptr(), kp.data_ptr(), float(keep),
+                                  mask.row_start.data_ptr(), mask.row_count.data_ptr(), mask.col_idx.data_ptr(),
+                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                  _stream(stream)), "rf2_predict_mask")
+    return mask
+
+
+def block_sparse_attn(geom: Geometry, qp, kp, vp, mask: BlockMask, out: torch.Tensor | None = None,
+                      lse: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _check_qkv(geom, qp, kp, vp)
+    out = torch.empty_like(qp) if out is None else out
+    _check_qkv(geom, out)
+    if lse is not None:
+        n = geom.frames * geom.height * geom.width
+        if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
+                and lse.numel() == geom.batch * geom.heads * n):
+            raise ValueError("lse must be a contiguous CUDA float32 tensor of B*H*N elements")
+    _check(lib().rf2_block_sparse_attn(ctypes.byref(geom), qp.data_ptr(), kp.data_ptr(), vp.data_ptr(),
+                                       mask.row_start.data_ptr(), mask.row_count.data_ptr(),
+                                       mask.col_idx.data_ptr(), out.data_ptr(),
+                                       lse.data_ptr() if lse is not None else None, _stream(stream)),
+           "rf2_block_sparse_attn")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronize and return (and clear) the device status word."""
+    return int(lib().rf2_device_status(_stream(stream)))
+
+
+def rainfusion_attention(geom: Geometry, q, k, v, keep: float, stream=None):
+    """The whole path for one attention call: permute Q/K/V, predict the block
+    mask, block-sparse attention, unpermute.  Returns (O, mask)."""
+    qp = permute(geom, q, stream=stream)
+    kp = permute(geom, k, stream=stream)
+    vp = permute(geom, v, stream=stream)
+    mask = predict_mask(geom, qp, kp, keep, stream=stream)
+    op = block_sparse_attn(geom, qp, kp, vp, mask, stream=stream)
+    return unpermute(geom, op, stream=stream), mask

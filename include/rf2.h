@@ -1,0 +1,139 @@
+/*
+ * rf2.h — C ABI of a B200 (sm_100a) implementation of the block-wise sparse
+ * attention of
+ *
+ *   "RainFusion2.0: Temporal-Spatial Awareness and Hardware-Efficient
+ *    Block-wise Sparse Attention" (arXiv 2512.24086).
+ *
+ * One attention call of a DiT layer is four library calls on one stream:
+ *
+ *   rf2_permute(Q), rf2_permute(K), rf2_permute(V)       section 3.3 + 3.4
+ *   rf2_predict_mask(Qp, Kp) -> block mask as CSR         section 3.2, eqs. (5)-(8) + 3.4
+ *   rf2_block_sparse_attn(Qp, Kp, Vp, mask) -> Op         section 3.1, eqs. (1)-(4)
+ *   rf2_unpermute(Op) -> O                                inverse of section 3.3
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Tensors are dense, row-major [batch, heads, N, head_dim] bf16 (d fastest),
+ *   N = frames * height * width in the model's [F, H, W] raster order, or the
+ *   permuted order for the "p" tensors.  Device pointers must be 16-byte
+ *   aligned.  The caller owns every buffer; the library never allocates
+ *   device memory, never synchronizes (except rf2_device_status) and keeps no
+ *   state between calls.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Every call is asynchronous on it and launches 1-2 kernels.
+ * - Arguments are validated on the host before anything is launched; an
+ *   invalid call returns an error status and launches nothing.  A failed
+ *   launch returns RF2_ERR_CUDA.  Kernels never trap: a bounded wait that
+ *   runs out records RF2_ERR_TIMEOUT in a device status word that
+ *   rf2_device_status reads back.
+ * - Blocks are 64 consecutive tokens of the permuted sequence; T_b =
+ *   ceil(N/64) and the last block may be short.
+ * - The geometry must be identical across the four calls of one invocation.
+ */
+#ifndef RF2_H
+#define RF2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RF2_OK = 0,
+    RF2_ERR_INVALID_ARGUMENT = 1,     /* null/misaligned pointer, bad size or ratio */
+    RF2_ERR_UNSUPPORTED = 2,          /* head_dim not 64/128, block not 64, too many blocks */
+    RF2_ERR_INSUFFICIENT_WORKSPACE = 3,
+    RF2_ERR_CUDA = 4,                 /* a CUDA runtime call or launch failed */
+    RF2_ERR_TIMEOUT = 5               /* a kernel's bounded wait ran out (device status) */
+} rf2_status;
+
+/* Problem geometry.  The window (win_t, win_h, win_w) is the 3D (video) or 2D
+ * (image, frames = 1) tile of section 3.3; the paper leaves its shape open, so
+ * it is a parameter.  Windows tile each segment from its origin and are cut
+ * short at the grid edge.  With first_frame_sink = 1 (section 3.4) frame 0 is
+ * moved behind frames 1..F-1, every query block holding a first-frame token
+ * keeps every key block, and every query block keeps every key block holding
+ * a first-frame token. */
+typedef struct {
+    int32_t batch, heads, head_dim;     /* head_dim in {64, 128} */
+    int32_t frames, height, width;      /* latent grid; frames = 1 for images */
+    int32_t win_t, win_h, win_w;        /* permutation window, each >= 1 */
+    int32_t block;                      /* query/key block size; 64 */
+    int32_t first_frame_sink;           /* 0 or 1 */
+} rf2_geometry;
+
+/* Derived sizes (rf2_query). */
+typedef struct {
+    int64_t num_tokens;          /* N */
+    int32_t num_blocks;          /* T_b = ceil(N / 64) */
+    int32_t n_keep;              /* top-n per query block: ceil(keep * T_b), in [1, T_b] */
+    int32_t sink_first;          /* first sink block, -1 when the sink is off */
+    int32_t row_capacity;        /* col_idx slots of a non-sink row: min(T_b, n_keep + sink blocks) */
+    int64_t num_rows;            /* batch * heads * T_b: length of row_start / row_count */
+    int64_t col_idx_capacity;    /* length of col_idx */
+    size_t  mask_workspace_bytes;/* scratch for rf2_predict_mask (block means, fp32) */
+} rf2_sizes;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* rf2_status_string(int status);
+
+/* Sizes for a geometry and keep ratio (the fraction of key blocks each query
+ * block keeps before the sink is added: 0.2 = "80% sparsity").  Host only.
+ * Returns RF2_ERR_INVALID_ARGUMENT / RF2_ERR_UNSUPPORTED for bad input. */
+int rf2_query(const rf2_geometry* geom, double keep_ratio, rf2_sizes* out);
+
+/* The window permutation of sections 3.3-3.4 as a host table:
+ * perm[p] = [F,H,W] raster index of the token placed at permuted position p.
+ * perm must hold N int32.  Host only; no device work. */
+int rf2_permutation_index(const rf2_geometry* geom, int32_t* perm);
+
+/* Xp[b,h,p,:] = X[b,h,perm[p],:] — gathers every (b, h) slice into window
+ * order (sections 3.3-3.4).  X and Xp must not overlap.  Pure copy: bit exact. */
+int rf2_permute(const rf2_geometry* geom, const void* x_bf16, void* xp_bf16, void* stream);
+
+/* X[b,h,perm[p],:] = Xp[b,h,p,:] — the inverse of rf2_permute, returning the
+ * attention output to the model's [F,H,W] order.  Bit exact. */
+int rf2_unpermute(const rf2_geometry* geom, const void* xp_bf16, void* x_bf16, void* stream);
+
+/* Online block-mask prediction (section 3.2, eqs. (5)-(8), and section 3.4).
+ *   q^_i = mean of the valid rows of query block i (fp32), likewise k^_j;
+ *   S^_ij = q^_i . k^_j / sqrt(d) (fp32);
+ *   a non-sink row keeps its n_keep largest S^_ij (equal scores: lower j
+ *   first) plus every sink column; a sink row keeps every column.
+ * Output is one CSR row per (b, h, i), r = (b*heads + h)*T_b + i:
+ *   row_start[r]  closed-form offset into col_idx (rows are laid out at
+ *                 their capacity, so col_idx may have gaps),
+ *   row_count[r]  number of kept key blocks,
+ *   col_idx[row_start[r] .. + row_count[r]) kept key blocks, ascending.
+ * row_start/row_count hold num_rows int32, col_idx col_idx_capacity int32,
+ * workspace at least mask_workspace_bytes (device, 16-byte aligned); its
+ * contents on entry do not matter.  qp/kp are the permuted Q and K. */
+int rf2_predict_mask(const rf2_geometry* geom, const void* qp_bf16, const void* kp_bf16,
+                     double keep_ratio, int32_t* row_start, int32_t* row_count, int32_t* col_idx,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Block-sparse FlashAttention forward (section 3.1): for every query block i,
+ * O_i = softmax(Q_i K_J^T / sqrt(d)) V_J over the key blocks J kept in row i
+ * of the CSR mask (eqs. (1)-(4); Q_i K_j^T and P_ij V_j are skipped when
+ * M_ij = 0).  bf16 operands, fp32 accumulation and fp32 softmax, P rounded to
+ * bf16 as the operand of the PV product.  op receives bf16 [B,H,N,d]; lse,
+ * when not NULL, receives the natural-log row sums fp32 [B,H,N].  Every row
+ * must keep at least one key block; col_idx entries must lie in [0, T_b) and
+ * ascend within a row (as rf2_predict_mask writes them). */
+int rf2_block_sparse_attn(const rf2_geometry* geom, const void* qp_bf16, const void* kp_bf16,
+                          const void* vp_bf16, const int32_t* row_start, const int32_t* row_count,
+                          const int32_t* col_idx, void* op_bf16, float* lse, void* stream);
+
+/* Synchronizes `stream`, then returns and clears the device status word of
+ * the calling thread's current device: RF2_OK, or RF2_ERR_TIMEOUT if a
+ * kernel's bounded wait ran out since the last call. */
+int rf2_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RF2_H */

@@ -1,0 +1,132 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+that include/rf2.h declares, computes the documented sizes, rejects invalid
+calls on the host before any launch, and its host permutation table (the same
+closed form the kernels use) equals the oracle's sort-based definition."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from image_dits_b200 import build as rf2_build
+from image_dits_b200 import rf2
+from image_dits_b200.workload import WORKLOADS, random_grid_case
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    rf2_build.build()
+    return rf2.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "rf2.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rf2_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_match_header(L):
+    declared = _declared()
+    assert declared == sorted(rf2.EXPORTED)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert rf2.status_string(s)
+    assert rf2.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_query_matches_oracle_readings(L, name):
+    wl = WORKLOADS[name]
+    sz = rf2.query(rf2.geometry_of(wl), wl.keep)
+    N = wl.num_tokens
+    assert sz.num_tokens == N
+    assert sz.num_blocks == oracle.num_blocks(N)
+    assert sz.n_keep == oracle.keep_count(wl.keep, sz.num_blocks)
+    assert sz.sink_first == oracle.sink_start(wl.frames, wl.height, wl.width, wl.sink)
+    Tb = sz.num_blocks
+    n_sink = 0 if sz.sink_first < 0 else Tb - sz.sink_first
+    assert sz.row_capacity == min(Tb, sz.n_keep + n_sink)
+    BH = wl.batch * wl.heads
+    assert sz.num_rows == BH * Tb
+    s0 = Tb if sz.sink_first < 0 else sz.sink_first
+    assert sz.col_idx_capacity == BH * (s0 * sz.row_capacity + (Tb - s0) * Tb)
+    assert sz.mask_workspace_bytes == 2 * BH * Tb * wl.head_dim * 4
+
+
+def test_keep_ratio_matches_oracle(L):
+    g = rf2.make_geometry(1, 1, 128, 21, 45, 80, 4, 4, 4, True)
+    for keep in (1.0, 0.5, 0.2, 0.1, 0.05, 0.3333, 1e-6, 0.9999):
+        assert rf2.query(g, keep).n_keep == oracle.keep_count(keep, 1182)
+
+
+def test_permutation_index_matches_oracle(L):
+    rng = np.random.default_rng(0)
+    cases = [random_grid_case(rng) for _ in range(250)]
+    cases += [(21, 45, 80, 4, 4, 4, True), (21, 30, 52, 4, 4, 4, True), (1, 64, 64, 1, 8, 8, False),
+              (4, 16, 16, 1, 8, 8, True), (5, 7, 9, 8, 9, 10, True)]
+    for (T, H, W, wt, wh, ww, sink) in cases:
+        g = rf2.make_geometry(1, 1, 64, T, H, W, wt, wh, ww, sink)
+        assert np.array_equal(rf2.permutation_index(g), oracle.permutation(T, H, W, wt, wh, ww, sink)), \
+            (T, H, W, wt, wh, ww, sink)
+
+
+def _status(fn, *args):
+    return fn(*args)
+
+
+def test_host_validation(L):
+    good = rf2.make_geometry(1, 2, 64, 4, 16, 16, 1, 8, 8, True)
+    fake = ctypes.c_void_p(0x10000)            # aligned, never dereferenced: validation fails first
+    G = ctypes.byref
+    bad_dim = rf2.make_geometry(1, 2, 96, 4, 16, 16, 1, 8, 8, True)
+    bad_blk = rf2.make_geometry(1, 2, 64, 4, 16, 16, 1, 8, 8, True, block=32)
+    bad_win = rf2.make_geometry(1, 2, 64, 4, 16, 16, 0, 8, 8, True)
+    bad_sink = rf2.make_geometry(1, 2, 64, 4, 16, 16, 1, 8, 8, True)
+    bad_sink.first_frame_sink = 2
+    huge = rf2.make_geometry(1, 1, 64, 100, 64, 64, 1, 8, 8, False)    # T_b > 4096
+    sz = rf2.Sizes()
+    assert L.rf2_query(G(good), 0.5, G(sz)) == rf2.RF2_OK
+    assert L.rf2_query(G(good), 0.0, G(sz)) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_query(G(good), 1.5, G(sz)) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_query(G(good), float("nan"), G(sz)) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_query(None, 0.5, G(sz)) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_query(G(good), 0.5, None) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_query(G(bad_dim), 0.5, G(sz)) == rf2.RF2_ERR_UNSUPPORTED
+    assert L.rf2_query(G(bad_blk), 0.5, G(sz)) == rf2.RF2_ERR_UNSUPPORTED
+    assert L.rf2_query(G(huge), 0.5, G(sz)) == rf2.RF2_ERR_UNSUPPORTED
+    assert L.rf2_query(G(bad_win), 0.5, G(sz)) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_query(G(bad_sink), 0.5, G(sz)) == rf2.RF2_ERR_INVALID_ARGUMENT
+    # permute / unpermute
+    for fn in (L.rf2_permute, L.rf2_unpermute):
+        assert fn(G(good), None, fake, None) == rf2.RF2_ERR_INVALID_ARGUMENT
+        assert fn(G(good), fake, None, None) == rf2.RF2_ERR_INVALID_ARGUMENT
+        assert fn(G(good), ctypes.c_void_p(0x10008), ctypes.c_void_p(0x20000), None) == rf2.RF2_ERR_INVALID_ARGUMENT
+        assert fn(G(good), fake, fake, None) == rf2.RF2_ERR_INVALID_ARGUMENT      # in place
+        assert fn(G(bad_dim), fake, ctypes.c_void_p(0x20000), None) == rf2.RF2_ERR_UNSUPPORTED
+    # predict_mask
+    L.rf2_query(G(good), 0.5, G(sz))
+    ws_small = sz.mask_workspace_bytes - 1
+    assert L.rf2_predict_mask(G(good), fake, fake, 0.5, fake, fake, fake, fake, ws_small, None) == \
+        rf2.RF2_ERR_INSUFFICIENT_WORKSPACE
+    assert L.rf2_predict_mask(G(good), fake, fake, 0.0, fake, fake, fake, fake, 1 << 30, None) == \
+        rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_predict_mask(G(good), None, fake, 0.5, fake, fake, fake, fake, 1 << 30, None) == \
+        rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_predict_mask(G(good), fake, fake, 0.5, fake, fake, fake, ctypes.c_void_p(0x10004), 1 << 30,
+                              None) == rf2.RF2_ERR_INVALID_ARGUMENT
+    # block_sparse_attn
+    assert L.rf2_block_sparse_attn(G(good), fake, fake, None, fake, fake, fake, fake, None, None) == \
+        rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_block_sparse_attn(G(good), fake, fake, fake, fake, fake, fake, fake, ctypes.c_void_p(0x10002),
+                                   None) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_block_sparse_attn(G(bad_dim), fake, fake, fake, fake, fake, fake, fake, None, None) == \
+        rf2.RF2_ERR_UNSUPPORTED
+    assert L.rf2_permutation_index(G(good), None) == rf2.RF2_ERR_INVALID_ARGUMENT

@@ -1,0 +1,179 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the oracle on
+the same seeded inputs.
+
+- permutation and unpermutation: bit exact;
+- block mask: bit exact outside the 1e-5 tie band around each row's threshold;
+- attention output under the GPU's mask: max-abs <= 2e-2, mean-abs <= 2e-3.
+Sizes span several tiles with ragged tails; the video workloads at full size
+are compared in full for the permutation and the mask, and on sampled query
+blocks for the attention output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from image_dits_b200 import build as rf2_build
+from image_dits_b200 import rf2
+from image_dits_b200.workload import WORKLOADS, Workload, make_qkv
+from parity import (ATTN_MAX_ABS, ATTN_MEAN_ABS, attention_errors, bits, check_csr, compare_masks, run_path)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    rf2_build.build()
+    rf2.lib()
+    yield
+    torch.cuda.synchronize()
+
+
+def _perm_of(wl):
+    return oracle.permutation(wl.frames, wl.height, wl.width, wl.win_t, wl.win_h, wl.win_w, wl.sink)
+
+
+def _small_cases():
+    """(name, Workload) small geometries: ragged tails, odd block counts, N < 64,
+    single frame with sink, windows larger than the grid, d = 64 and 128."""
+    W = Workload
+    return [
+        ("tiny", WORKLOADS["tiny"]),
+        ("ragged_d128", W("r1", 1, 3, 128, 3, 7, 9, 2, 4, 4, 0.3, True, (44, 42, 42))),
+        ("ragged_d64_nosink", W("r2", 2, 1, 64, 2, 13, 11, 2, 3, 5, 0.5, False, (24, 20, 20))),
+        ("one_block", W("r3", 1, 2, 64, 1, 5, 7, 1, 2, 2, 0.5, True, (0, 32, 32))),
+        ("single_frame_sink", W("r4", 1, 2, 128, 1, 16, 20, 1, 8, 8, 0.25, True, (0, 64, 64))),
+        ("big_window", W("r5", 1, 1, 128, 5, 9, 10, 8, 16, 16, 0.2, True, (44, 42, 42))),
+        ("keep_one", W("r6", 1, 2, 128, 3, 16, 16, 1, 8, 8, 0.01, True, (44, 42, 42))),
+        ("keep_all", W("r7", 1, 2, 64, 2, 12, 16, 2, 4, 4, 1.0, True, (24, 20, 20))),
+        ("odd_blocks", W("r8", 1, 2, 128, 1, 24, 40, 1, 8, 8, 0.4, False, (0, 64, 64))),
+    ]
+
+
+@pytest.mark.parametrize("name,wl", _small_cases())
+def test_small_case_parity(name, wl):
+    q, k, v = make_qkv(wl, "cuda", seed=7)
+    g = rf2.geometry_of(wl)
+    out = run_path(g, q, k, v, wl.keep, lse=True)
+    perm = _perm_of(wl)
+    # permutation: bit exact, and unpermute(permute(x)) == x
+    assert np.array_equal(bits(out["qp"]), oracle.permute(bits(q), perm))
+    assert np.array_equal(bits(out["vp"]), oracle.permute(bits(v), perm))
+    assert torch.equal(rf2.unpermute(g, out["qp"]).view(torch.int16), q.view(torch.int16))
+    # mask
+    sz = out["mask"].sizes
+    check_csr(out["mask"], sz.sink_first)
+    dense = out["mask"].dense()
+    compare_masks(dense, bits(out["qp"]), bits(out["kp"]), wl.keep, wl.frames, wl.height, wl.width, wl.sink)
+    # attention under the GPU's mask, and the unpermuted output
+    e = attention_errors(out["op"], bits(out["qp"]), bits(out["kp"]), bits(out["vp"]), dense, lse=out["lse"])
+    assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, e
+    assert e["lse_max_abs"] <= 1e-3, e
+    assert np.array_equal(bits(out["o"]), oracle.unpermute(bits(out["op"]), perm))
+
+
+def test_image_parity():
+    wl = WORKLOADS["image"]
+    q, k, v = make_qkv(wl, "cuda", seed=0)
+    g = rf2.geometry_of(wl)
+    out = run_path(g, q, k, v, wl.keep)
+    perm = _perm_of(wl)
+    assert np.array_equal(bits(out["kp"]), oracle.permute(bits(k), perm))
+    check_csr(out["mask"], -1)
+    dense = out["mask"].dense()
+    compare_masks(dense, bits(out["qp"]), bits(out["kp"]), wl.keep, 1, wl.height, wl.width, False)
+    Tb = wl.num_blocks
+    items = [(bh, i) for bh in (0, 11, 23) for i in range(Tb)]
+    e = attention_errors(out["op"], bits(out["qp"]), bits(out["kp"]), bits(out["vp"]), dense, items=items)
+    assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, e
+
+
+def test_keep_all_equals_dense_attention():
+    """keep = 1 selects every block: the output is dense softmax attention, and
+    unpermuting it gives dense attention in the model's order."""
+    wl = Workload("dense", 1, 2, 128, 2, 10, 13, 2, 4, 4, 1.0, False, (44, 42, 42))
+    q, k, v = make_qkv(wl, "cuda", seed=3)
+    g = rf2.geometry_of(wl)
+    out = run_path(g, q, k, v, 1.0)
+    assert out["mask"].kept_pairs() == wl.heads * wl.num_blocks ** 2
+    ref = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double())
+    err = (out["o"].double() - ref).abs()
+    assert err.max().item() <= ATTN_MAX_ABS and err.mean().item() <= ATTN_MEAN_ABS
+
+
+def test_constant_value_rows():
+    """With V constant along the sequence every output row equals that row."""
+    wl = Workload("const", 1, 2, 128, 3, 9, 11, 2, 4, 4, 0.3, True, (44, 42, 42))
+    q, k, v = make_qkv(wl, "cuda", seed=5)
+    v = v[:, :, :1, :].expand_as(v).contiguous()
+    out = run_path(rf2.geometry_of(wl), q, k, v, wl.keep)
+    err = (out["o"].float() - v.float()).abs().max().item()
+    assert err <= 2 ** -7 * v.float().abs().max().item() + 1e-6
+
+
+def test_deterministic():
+    wl = WORKLOADS["tiny"]
+    q, k, v = make_qkv(wl, "cuda", seed=11)
+    g = rf2.geometry_of(wl)
+    a = run_path(g, q, k, v, wl.keep)
+    b = run_path(g, q, k, v, wl.keep)
+    assert torch.equal(a["mask"].row_count, b["mask"].row_count)
+    assert np.array_equal(a["mask"].dense(), b["mask"].dense())
+    assert torch.equal(a["o"].view(torch.int16), b["o"].view(torch.int16))
+
+
+def test_random_geometries():
+    rng = np.random.default_rng(21)
+    for it in range(12):
+        T, H, W = int(rng.integers(1, 4)), int(rng.integers(2, 20)), int(rng.integers(2, 20))
+        d = int(rng.choice([64, 128]))
+        rope = (0, d // 2, d // 2) if T == 1 else ((24, 20, 20) if d == 64 else (44, 42, 42))
+        wl = Workload(f"rand{it}", 1, int(rng.integers(1, 3)), d, T, H, W, int(rng.integers(1, 4)),
+                      int(rng.integers(1, 9)), int(rng.integers(1, 9)), float(rng.choice([0.1, 0.3, 0.5, 0.8])),
+                      bool(rng.integers(0, 2)), rope)
+        q, k, v = make_qkv(wl, "cuda", seed=it)
+        g = rf2.geometry_of(wl)
+        out = run_path(g, q, k, v, wl.keep)
+        assert np.array_equal(bits(out["qp"]), oracle.permute(bits(q), _perm_of(wl))), wl
+        dense = out["mask"].dense()
+        check_csr(out["mask"], out["mask"].sizes.sink_first)
+        compare_masks(dense, bits(out["qp"]), bits(out["kp"]), wl.keep, T, H, W, wl.sink)
+        e = attention_errors(out["op"], bits(out["qp"]), bits(out["kp"]), bits(out["vp"]), dense)
+        assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, (wl, e)
+
+
+def _full_size(name, n_random_blocks, n_sink_blocks):
+    wl = WORKLOADS[name]
+    q, k, v = make_qkv(wl, "cuda", seed=0)
+    g = rf2.geometry_of(wl)
+    out = run_path(g, q, k, v, wl.keep)
+    perm = _perm_of(wl)
+    qp_b, kp_b, vp_b = bits(out["qp"]), bits(out["kp"]), bits(out["vp"])
+    assert np.array_equal(qp_b, oracle.permute(bits(q), perm))
+    assert np.array_equal(vp_b, oracle.permute(bits(v), perm))
+    del q, k, v
+    sz = out["mask"].sizes
+    dense = out["mask"].dense()
+    excluded, compared = compare_masks(dense, qp_b, kp_b, wl.keep, wl.frames, wl.height, wl.width, wl.sink)
+    assert excluded <= 1e-4 * compared
+    rng = np.random.default_rng(1)
+    Tb = sz.num_blocks
+    BH = wl.heads
+    items = [(int(rng.integers(0, BH)), int(rng.integers(0, sz.sink_first))) for _ in range(n_random_blocks)]
+    items += [(int(rng.integers(0, BH)), int(rng.integers(sz.sink_first, Tb))) for _ in range(n_sink_blocks)]
+    items += [(BH - 1, Tb - 1), (0, Tb - 1)]             # ragged last block
+    e = attention_errors(out["op"], qp_b, kp_b, vp_b, dense, items=items)
+    assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, e
+    assert np.array_equal(bits(out["o"][:, :2]), oracle.unpermute(bits(out["op"][:, :2]), perm))
+
+
+def test_video480p_full_size():
+    _full_size("video480p", 48, 4)
+
+
+def test_video720p_full_size():
+    _full_size("video720p", 48, 4)
+
+
+def test_device_status_clean():
+    assert rf2.device_status() == rf2.RF2_OK
