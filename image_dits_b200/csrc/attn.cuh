@@ -59,7 +59,7 @@ struct AttnCfg {
     static constexpr uint32_t OFF_LIST = OFF_V + STAGES * KV_BYTES;
     static constexpr uint32_t CONTROL_BYTES = 256;
     // The list is padded to 16 bytes so the control block (mbarriers) stays aligned.
-    static size_t list_bytes(int Tb) { return ((size_t)Tb * 4 + 15) & ~(size_t)15; }
+    __host__ __device__ static size_t list_bytes(int Tb) { return ((size_t)Tb * 4 + 15) & ~(size_t)15; }
     static size_t smem_bytes(int Tb) { return 1024 + OFF_LIST + list_bytes(Tb) + CONTROL_BYTES; }
 };
 
