@@ -136,6 +136,24 @@ class ClockSampler:
                 "power_w_max": max(power)}
 
 
+def combine_over_ranks(ms_step, attn_ms, e2e_ms, flops, dist=None, device="cpu"):
+    """Whole-job numbers: every time is the max over ranks, the work is the sum."""
+    vals = torch.tensor([ms_step, attn_ms, e2e_ms, flops], dtype=torch.float64, device=device)
+    if dist is not None:
+        mx = vals.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = vals.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        vals = torch.cat([mx[:3], sm[3:]])
+    v = vals.cpu().tolist()
+    return {"ms_step": v[0], "attn_ms": v[1], "e2e_ms": v[2], "flops": v[3]}
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own batch element: independent seeded inputs."""
+    return 1000 * rank
+
+
 def cpu_info():
     model = "unknown"
     try:
@@ -259,7 +277,7 @@ def main():
     rf2.lib()
 
     g = rf2.geometry_of(wl)
-    q, k, v = make_qkv(wl, dev, seed=1000 * rank)
+    q, k, v = make_qkv(wl, dev, seed=rank_seed(rank))
     qp, kp, vp, op, o = (torch.empty_like(q) for _ in range(5))
     mask, ws = rf2.alloc_mask(g, wl.keep, dev)
     stream = torch.cuda.current_stream()
@@ -339,20 +357,11 @@ def main():
         e2e_ms = e0.elapsed_time(e1) / args.steps
         e2e = {"ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2}
 
-    # ---- max over ranks
+    # ---- max over ranks (times), sum over ranks (work)
     ms_step = total_ms / args.steps
-    vals = torch.tensor([ms_step, stage_ms["block_sparse_attn"], e2e["ms_per_step"] if e2e else 0.0, flops],
-                        dtype=torch.float64, device=dev)
-    if dist:
-        mx = vals.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = vals.clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        ms_step_all, attn_ms_all, e2e_ms_all = float(mx[0]), float(mx[1]), float(mx[2])
-        flops_all = float(sm[3])
-    else:
-        ms_step_all, attn_ms_all, e2e_ms_all, flops_all = ms_step, stage_ms["block_sparse_attn"], \
-            (e2e["ms_per_step"] if e2e else 0.0), flops
+    comb = combine_over_ranks(ms_step, stage_ms["block_sparse_attn"], e2e["ms_per_step"] if e2e else 0.0, flops,
+                              dist, dev)
+    ms_step_all, attn_ms_all, e2e_ms_all, flops_all = comb["ms_step"], comb["attn_ms"], comb["e2e_ms"], comb["flops"]
 
     peaks, peak_src = load_peaks()
     attn_tf = flops / (stage_ms["block_sparse_attn"] * 1e-3) / 1e12

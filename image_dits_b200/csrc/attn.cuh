@@ -5,8 +5,8 @@
 // Work unit: one CTA computes two adjacent 64-row query blocks (2p, 2p+1) of
 // one (batch, head) as a single M = 128 tile, the native row count of a
 // cta_group::1 tcgen05 MMA.  The key blocks it visits are the sorted union of
-// the two blocks' CSR rows; each union entry carries one "kept" bit per
-// query block, and the rows of a block that did not keep key block j are
+// the two blocks' CSR rows (bitmap union, so rows need not even be sorted);
+// each union entry carries one "kept" bit per query block, and the rows of a block that did not keep key block j are
 // masked to -inf in the softmax (their P is exactly 0), so every row sees
 // exactly its own kept blocks.
 //
@@ -71,7 +71,6 @@ struct __align__(16) AttnCtl {
     uint64_t o_done, o_final, drain;
     uint32_t tmem_base;
     int32_t list_len;
-    int32_t dups;
     int32_t abort;
 };
 
@@ -90,16 +89,6 @@ struct AttnArgs {
     int32_t sink_pairs;     // pairs holding a sink block: scheduled first in each head
     float scale_log2;       // log2(e) / sqrt(D)
 };
-
-__device__ __forceinline__ int lower_bound_smem(const int32_t* a, int n, int32_t v)
-{
-    int lo = 0, hi = n;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (a[mid] < v) lo = mid + 1; else hi = mid;
-    }
-    return lo;
-}
 
 template <int D>
 __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 2)
@@ -141,7 +130,6 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_init(smem_u32(&ctl->o_done), 1);
         mbar_init(smem_u32(&ctl->o_final), 1);
         mbar_init(smem_u32(&ctl->drain), 1);
-        ctl->dups = 0;
         ctl->abort = 0;
         fence_mbar_init();
     }
@@ -154,50 +142,81 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_alloc(smem_u32(&ctl->tmem_base), Cfg::TM_COLS);
         tmem_relinquish();
     }
-    // The two rows are staged in the (still unused) K/V rings.
-    int32_t* rowA = reinterpret_cast<int32_t*>(base + Cfg::OFF_K);
-    int32_t* rowB = rowA + Tb;
-    const int64_t rA = bh * Tb + qb0;
-    const int lenA = min(max(args.row_count[rA], 0), Tb);
-    const int lenB = has_b ? min(max(args.row_count[rA + 1], 0), Tb) : 0;
-    {
-        const int32_t* srcA = args.col_idx + args.row_start[rA];
-        for (int e = tid; e < lenA; e += Cfg::THREADS) rowA[e] = srcA[e];
-        if (has_b) {
-            const int32_t* srcB = args.col_idx + args.row_start[rA + 1];
-            for (int e = tid; e < lenB; e += Cfg::THREADS) rowB[e] = srcB[e];
-        }
-    }
+    // Union of the two CSR rows as bitmaps (one bit per key block and query
+    // block), built in the still unused K/V rings, then compacted in
+    // ascending order: a word's entries start at the popcount of all earlier
+    // words of (A | B).
+    const int W = (Tb + 31) >> 5;                          // <= 128 words
+    uint32_t* bmA = reinterpret_cast<uint32_t*>(base + Cfg::OFF_K);
+    uint32_t* bmB = bmA + W;
+    int32_t* word_off = reinterpret_cast<int32_t*>(bmB + W);
+    for (int w = tid; w < 2 * W; w += Cfg::THREADS) bmA[w] = 0u;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
+    const int64_t rA = bh * Tb + qb0;
     {
-        // Merge by rank: an entry's place in the union is its index in its own
-        // row plus the number of smaller entries in the other row.
-        int dups = 0;
+        const int lenA = min(max(args.row_count[rA], 0), Tb);
+        const int32_t* srcA = args.col_idx + args.row_start[rA];
         for (int e = tid; e < lenA; e += Cfg::THREADS) {
-            const int32_t a = rowA[e];
-            const int pb = lower_bound_smem(rowB, lenB, a);
-            const int in_b = (pb < lenB && rowB[pb] == a) ? 1 : 0;
-            if (e + pb < Tb) list[e + pb] = (a & 0x3fffffff) | (1 << 30) | (in_b << 31);
+            const int32_t j = srcA[e];
+            if (j >= 0 && j < Tb) atomicOr(&bmA[j >> 5], 1u << (j & 31));
         }
-        for (int e = tid; e < lenB; e += Cfg::THREADS) {
-            const int32_t b = rowB[e];
-            const int pa = lower_bound_smem(rowA, lenA, b);
-            if (pa < lenA && rowA[pa] == b) { ++dups; continue; }
-            if (e + pa < Tb) list[e + pa] = (b & 0x3fffffff) | (1 << 31);
+        if (has_b) {
+            const int lenB = min(max(args.row_count[rA + 1], 0), Tb);
+            const int32_t* srcB = args.col_idx + args.row_start[rA + 1];
+            for (int e = tid; e < lenB; e += Cfg::THREADS) {
+                const int32_t j = srcB[e];
+                if (j >= 0 && j < Tb) atomicOr(&bmB[j >> 5], 1u << (j & 31));
+            }
         }
-        if (dups) atomicAdd(&ctl->dups, dups);
     }
     __syncthreads();
-    const int L = min(lenA + lenB - ctl->dups, Tb);
+    if (warp == 0) {
+        // exclusive scan of per-word popcounts, 4 consecutive words per lane
+        int cnt[4];
+        int local = 0;
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int w = lane * 4 + k;
+            cnt[k] = (w < W) ? __popc(bmA[w] | bmB[w]) : 0;
+            local += cnt[k];
+        }
+        int incl = local;
+        #pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        int run = incl - local;
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int w = lane * 4 + k;
+            if (w < W) word_off[w] = run;
+            run += cnt[k];
+        }
+        if (lane == 31) ctl->list_len = incl;
+    }
+    __syncthreads();
+    for (int w = tid; w < W; w += Cfg::THREADS) {
+        const uint32_t a = bmA[w], b = bmB[w];
+        uint32_t u = a | b;
+        int pos = word_off[w];
+        while (u) {
+            const int bit = __ffs(u) - 1;
+            u &= u - 1;
+            list[pos++] = (w * 32 + bit) | (int32_t)(((a >> bit) & 1u) << 30) | (int32_t)(((b >> bit) & 1u) << 31);
+        }
+    }
+    __syncthreads();
+    const int L = ctl->list_len;
     volatile int* abort = &ctl->abort;
 
     if (warp == Cfg::PRODUCER_WARP) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            fence_proxy_async_smem();   // the rings held the row lists (generic writes)
+            fence_proxy_async_smem();   // the rings held the row bitmaps (generic accesses)
             const uint32_t q_s = base_u32 + Cfg::OFF_Q;
             mbar_arrive_expect_tx(smem_u32(&ctl->q_full), Cfg::Q_BYTES);
             for (int c = 0; c < Cfg::KCH; ++c)
