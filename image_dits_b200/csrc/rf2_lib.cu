@@ -9,6 +9,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "rf2.h"
 #include "attn.cuh"
 #include "geometry.cuh"
@@ -221,6 +223,33 @@ static int launch_select(const Checked& c, const MaskGeo& mg, const float* means
     return launch_status();
 }
 
+// ------------------------------------------------------------------------
+// Fixed device scratch for rf2_predict_mask_static (callers that cannot
+// allocate).  Every device that loads this library holds these 64 MiB until
+// the process exits.  In host code `g_static_scratch` only names a host-side
+// stand-in, so its device address is looked up once per device.
+constexpr size_t kStaticScratchBytes = (size_t)64 << 20;
+static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+static float* g_static_scratch_addr[kMaxDevices];
+static std::mutex g_static_scratch_mutex;
+
+// Device address of the scratch on the current device (set-up on first use).
+static int static_scratch(float** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RF2_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    if (!g_static_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return RF2_ERR_CUDA;
+        g_static_scratch_addr[dev] = static_cast<float*>(p);
+    }
+    *out = g_static_scratch_addr[dev];
+    return RF2_OK;
+}
+
 }  // namespace rf2
 
 using namespace rf2;
@@ -316,6 +345,43 @@ int rf2_block_sparse_attn(const rf2_geometry* geom, const void* qp, const void* 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return (c.D == 128) ? launch_attn<128>(c, mg, qp, kp, vp, row_start, row_count, col_idx, op, lse, s)
                         : launch_attn<64>(c, mg, qp, kp, vp, row_start, row_count, col_idx, op, lse, s);
+}
+
+int rf2_predict_mask_static(const rf2_geometry* geom, const void* qp, const void* kp, double keep_ratio,
+                            int32_t* row_start, int32_t* row_count, int32_t* col_idx, void* stream)
+{
+    Checked c;
+    MaskGeo mg;
+    rf2_sizes sz;
+    const int st = sizes_for(geom, keep_ratio, c, mg, &sz);
+    if (st != RF2_OK) return st;
+    if (!qp || !kp || !row_start || !row_count || !col_idx) return RF2_ERR_INVALID_ARGUMENT;
+    if (!aligned16(qp) || !aligned16(kp) || !aligned16(row_start) || !aligned16(row_count) || !aligned16(col_idx))
+        return RF2_ERR_INVALID_ARGUMENT;
+    if (sz.mask_workspace_bytes > kStaticScratchBytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    float* means = nullptr;
+    const int ss = static_scratch(&means);
+    if (ss != RF2_OK) return ss;
+    // The block means fill every scratch element the select kernel reads, so
+    // nothing left from an earlier call needs clearing.
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t warps = 2 * c.BH * c.Tb;
+    const unsigned grid = (unsigned)((warps + 7) / 8);
+    if (c.D == 128)
+        block_mean_kernel<128><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
+                                                     reinterpret_cast<const uint4*>(kp), means, c.N, c.Tb, c.BH);
+    else
+        block_mean_kernel<64><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
+                                                    reinterpret_cast<const uint4*>(kp), means, c.N, c.Tb, c.BH);
+    int r = launch_status();
+    if (r != RF2_OK) return r;
+    if (c.Tb <= 2048)
+        r = (c.D == 128) ? launch_select<128, 16>(c, mg, means, row_start, row_count, col_idx, s)
+                         : launch_select<64, 16>(c, mg, means, row_start, row_count, col_idx, s);
+    else
+        r = (c.D == 128) ? launch_select<128, 8>(c, mg, means, row_start, row_count, col_idx, s)
+                         : launch_select<64, 8>(c, mg, means, row_start, row_count, col_idx, s);
+    return r;
 }
 
 int rf2_device_status(void* stream)

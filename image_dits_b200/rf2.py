@@ -26,7 +26,7 @@ RF2_ERR_TIMEOUT = 5
 # Every entry point declared in include/rf2.h.
 EXPORTED = (
     "rf2_status_string", "rf2_query", "rf2_permutation_index", "rf2_permute", "rf2_unpermute",
-    "rf2_predict_mask", "rf2_block_sparse_attn", "rf2_device_status",
+    "rf2_predict_mask", "rf2_predict_mask_static", "rf2_block_sparse_attn", "rf2_device_status",
 )
 
 
@@ -74,6 +74,7 @@ def lib():
         L.rf2_permute.argtypes = [G, vp, vp, vp]
         L.rf2_unpermute.argtypes = [G, vp, vp, vp]
         L.rf2_predict_mask.argtypes = [G, vp, vp, f64, vp, vp, vp, vp, sz, vp]
+        L.rf2_predict_mask_static.argtypes = [G, vp, vp, f64, vp, vp, vp, vp]
         L.rf2_block_sparse_attn.argtypes = [G, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.rf2_device_status.argtypes = [vp]
         for name in EXPORTED:

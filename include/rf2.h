@@ -19,7 +19,7 @@
  *   permuted order for the "p" tensors.  Device pointers must be 16-byte
  *   aligned.  The caller owns every buffer; the library never allocates
  *   device memory, never synchronizes (except rf2_device_status) and keeps no
- *   state between calls.
+ *   state between calls (rf2_predict_mask_static's fixed scratch aside).
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   Every call is asynchronous on it and launches 1-2 kernels.
  * - Arguments are validated on the host before anything is launched; an
@@ -114,6 +114,30 @@ int rf2_unpermute(const rf2_geometry* geom, const void* xp_bf16, void* x_bf16, v
 int rf2_predict_mask(const rf2_geometry* geom, const void* qp_bf16, const void* kp_bf16,
                      double keep_ratio, int32_t* row_start, int32_t* row_count, int32_t* col_idx,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* rf2_predict_mask without a caller-supplied workspace: the same computation
+ * and outputs, with the block-mean scratch taken from a fixed 64 MiB array
+ * inside the library instead.  For callers that cannot allocate device
+ * memory themselves — for example code embedded in a host framework that
+ * owns the device allocator and hands out no workspace, or a latency-critical
+ * loop where cudaMalloc's implicit device synchronization is not acceptable.
+ * (The paper has no counterpart to this call; it exists only for such callers.)
+ * - Limit: 2*batch*heads*T_b*head_dim*4 bytes (rf2_sizes.mask_workspace_bytes)
+ *   must not exceed 64 MiB (67,108,864), i.e. batch*heads <= 55 at 720p
+ *   (75,600 tokens, d = 128); larger problems return
+ *   RF2_ERR_INSUFFICIENT_WORKSPACE and launch nothing (split the heads over
+ *   several calls, or use rf2_predict_mask).
+ * - Every GPU that loads the library holds the 64 MiB until the process exits.
+ * - The first call on a device looks up the array's device address (with that
+ *   device current) and caches it; make that first call before any stream
+ *   capture.  It allocates nothing, and calls no allocating routine.
+ * - All calls share the one array and it keeps the last call's contents;
+ *   nothing in it needs to start at zero, but calls that overlap on the GPU
+ *   (different streams, or different host threads on one device) race on it.
+ * Arguments, outputs and errors are otherwise those of rf2_predict_mask. */
+int rf2_predict_mask_static(const rf2_geometry* geom, const void* qp_bf16, const void* kp_bf16,
+                            double keep_ratio, int32_t* row_start, int32_t* row_count, int32_t* col_idx,
+                            void* stream);
 
 /* Block-sparse FlashAttention forward (section 3.1): for every query block i,
  * O_i = softmax(Q_i K_J^T / sqrt(d)) V_J over the key blocks J kept in row i
