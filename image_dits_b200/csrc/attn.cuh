@@ -3,28 +3,42 @@
 // M_ij = 0).
 //
 // Work unit: one CTA computes two adjacent 64-row query blocks (2p, 2p+1) of
-// one (batch, head) as a single M = 128 tile, the native row count of a
-// cta_group::1 tcgen05 MMA.  The key blocks it visits are the sorted union of
-// the two blocks' CSR rows (bitmap union, so rows need not even be sorted);
-// each union entry carries one "kept" bit per query block, and the rows of a block that did not keep key block j are
-// masked to -inf in the softmax (their P is exactly 0), so every row sees
-// exactly its own kept blocks.
+// one (batch, head) as a single M = 128 tile (a cta_group::1 tcgen05 MMA runs
+// at full rate only at M = 128; M = 64 runs at half rate).  It visits the
+// sorted union of the two blocks' CSR rows (built as bitmaps, so rows need
+// not even be sorted); each union entry carries one "kept" bit per query
+// block, and the rows of a block that did not keep key block j get no
+// probability mass from it (P exactly 0), so every row sees exactly its own
+// kept blocks.
 //
-// Roles (192 threads):
-//   warps 0-3  softmax + epilogue: thread r owns query row r, i.e. TMEM lane r
-//   warp 4     TMA producer: Q once, then K_j and V_j tiles of every visited
-//              key block into 2-stage rings (128-byte swizzled tiles)
-//   warp 5     MMA issuer (one thread):  S_t = Q K_t^T  (SS, M128 N64, into
-//              one of two TMEM S buffers) and O += P_t V_t (TS: P read from
-//              TMEM where softmax wrote it over S_t, V from shared memory)
-// TMEM: O (d fp32 columns) + two 64-column S/P buffers = 256 columns, so
-// two CTAs fit on an SM and one's softmax overlaps the other's MMAs.
+// A step covers two union entries (128 keys): S = Q [K_a; K_b]^T is one
+// M128 x N128 product (an N = 64 product leaves a third of the tensor pipe
+// idle), then O += P [V_a; V_b].
 //
-// Online softmax (eqs. (2)-(4)) in fp32 in the log2 domain.  The running max
-// m is only raised when a block's max exceeds it by more than 8 (a factor
-// 256), so O (in TMEM) is rarely rescaled; because O and l always use the
-// same m, the final O / l is unchanged.  Scale, exp2 and sums are fp32; P is
-// rounded to bf16 as the MMA operand.
+// Roles (256 threads, two CTAs per SM so that one CTA's softmax overlaps the
+// other's MMAs):
+//   warps 0-3  softmax + epilogue: thread r owns query row r = TMEM lane r
+//              and its full 128-column score row
+//   warp 4     MMA issuer (one thread)
+//   warp 5     TMA: Q once, then K of the step's first key block
+//   warp 6     TMA: K of the step's second key block
+//   warp 7     TMA: V of both key blocks
+// (one thread's TMA stream is served serially, so loads are spread over three
+// issuing warps).  Shared memory: Q 32 KB and one 32 KB K and V stage, all
+// 128-byte swizzled.  TMEM: O (d fp32 columns) and one 128-column S buffer;
+// P (bf16) is written over the first 64 columns of S and read by the PV
+// product straight from TMEM.  Per CTA the chain is S_t -> softmax_t -> PV_t
+// -> S_{t+1}; the tensor pipe serves the other CTA in between.
+//
+// Softmax (eqs. (2)-(4)) in fp32, log2 domain, per thread: pass 1 loads the
+// row's scores 32 columns at a time for the block max; pass 2 reloads them
+// (the next chunk's load in flight while the current one is exponentiated),
+// writes P in bf16 and accumulates the row sum.  The running max m is raised
+// (and O rescaled in TMEM) only when a step's max exceeds it by more than 8
+// (a factor 256); O and l always use the same m, so O / l is unchanged.  O
+// can be rescaled without waiting: PV_{t-1} was issued before S_t, so it has
+// completed once S_t has.  kExpEmu of every 32 exponentials per chunk run on
+// the FMA pipe (exp2_poly) instead of the SFU.
 //
 // Every wait on an mbarrier is bounded (ptx.cuh): on a timeout the CTA
 // raises a shared abort flag, every role leaves its loop, in-flight TMA loads
@@ -34,46 +48,48 @@
 #include "geometry.cuh"
 #include "ptx.cuh"
 
+#ifndef RF2_EXP2_EMU
+#define RF2_EXP2_EMU 0
+#endif
+
 namespace rf2 {
 
 template <int D>
 struct AttnCfg {
-    static constexpr int BM = 128;
-    static constexpr int BN = 64;
-    static constexpr int KCH = D / 64;                 // 128-byte column chunks per row
-    static constexpr int STAGES = 2;
-    static constexpr uint32_t Q_CHUNK = BM * 128;      // bytes of one 64-column chunk of Q
-    static constexpr uint32_t KV_CHUNK = BN * 128;
+    static constexpr int KCH = D / 64;                     // 128-byte column chunks per row
+    static constexpr uint32_t Q_CHUNK = 128 * 128;         // one 64-column chunk of Q (128 rows)
     static constexpr uint32_t Q_BYTES = Q_CHUNK * KCH;
-    static constexpr uint32_t KV_BYTES = KV_CHUNK * KCH;
+    static constexpr uint32_t K_CHUNK = 128 * 128;         // one chunk of the K stage: 128 key rows
+    static constexpr uint32_t KV_STAGE = 128 * D * 2;      // two 64-key blocks
+    static constexpr uint32_t V_BLOCK = 64 * D * 2;        // one key block of V: [chunk][64 rows]
     static constexpr uint32_t TM_O = 0;
-    static constexpr uint32_t TM_S = D;                // S/P buffer b at TM_S + 64*b
+    static constexpr uint32_t TM_S = 128;
     static constexpr uint32_t TM_COLS = 256;
-    static constexpr int THREADS = 192;
-    static constexpr int PRODUCER_WARP = 4;
-    static constexpr int MMA_WARP = 5;
-    // Shared memory: [align slack][Q][K ring][V ring][union list (Tb words)][control]
+    static constexpr int THREADS = 256;
+    static constexpr int MMA_WARP = 4;
+    static constexpr int KA_WARP = 5;
+    static constexpr int KB_WARP = 6;
+    static constexpr int V_WARP = 7;
+    // Shared memory: [align slack][Q][K stage][V stage][union list][control]
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = Q_BYTES;
-    static constexpr uint32_t OFF_V = OFF_K + STAGES * KV_BYTES;
-    static constexpr uint32_t OFF_LIST = OFF_V + STAGES * KV_BYTES;
+    static constexpr uint32_t OFF_V = OFF_K + KV_STAGE;
+    static constexpr uint32_t OFF_LIST = OFF_V + KV_STAGE;
     static constexpr uint32_t CONTROL_BYTES = 256;
-    // The list is padded to 16 bytes so the control block (mbarriers) stays aligned.
     __host__ __device__ static size_t list_bytes(int Tb) { return ((size_t)Tb * 4 + 15) & ~(size_t)15; }
-    static size_t smem_bytes(int Tb) { return 1024 + OFF_LIST + list_bytes(Tb) + CONTROL_BYTES; }
+    __host__ __device__ static size_t smem_bytes(int Tb) { return 1024 + OFF_LIST + list_bytes(Tb) + CONTROL_BYTES; }
 };
 
 struct __align__(16) AttnCtl {
     uint64_t q_full;
-    uint64_t k_full[2], k_empty[2];
-    uint64_t v_full[2], v_empty[2];
-    uint64_t s_full[2], p_full[2];
-    uint64_t o_done, o_final, drain;
+    uint64_t k_full, k_empty;
+    uint64_t v_full, v_empty;
+    uint64_t s_full, p_full;
+    uint64_t o_final, drain;
     uint32_t tmem_base;
     int32_t list_len;
     int32_t abort;
 };
-
 static_assert(sizeof(AttnCtl) <= 256, "control block must fit CONTROL_BYTES");
 
 struct AttnArgs {
@@ -90,10 +106,43 @@ struct AttnArgs {
     float scale_log2;       // log2(e) / sqrt(D)
 };
 
+// 32 scores of one row -> 16 packed bf16 pairs of P = 2^(s*sl2 - m), adding
+// the fp32 probabilities to sum4.  `nvalid` < 32 masks the tail columns.
+template <bool kMasked>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], float sl2, float neg_mu, int nvalid,
+                                          uint32_t (&pk)[16], float (&sum4)[4])
+{
+    #pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+        const float x0 = fmaf(__uint_as_float(s[c]), sl2, neg_mu);
+        const float x1 = fmaf(__uint_as_float(s[c + 1]), sl2, neg_mu);
+        float p0 = (c < RF2_EXP2_EMU) ? exp2_poly(x0) : ex2_approx(x0);
+        float p1 = (c + 1 < RF2_EXP2_EMU) ? exp2_poly(x1) : ex2_approx(x1);
+        if (kMasked) {
+            p0 = (c < nvalid) ? p0 : 0.f;
+            p1 = (c + 1 < nvalid) ? p1 : 0.f;
+        }
+        sum4[(c >> 1) & 3] += p0 + p1;
+        pk[c >> 1] = pack_bf16x2(p0, p1);
+    }
+}
+
+template <bool kMasked>
+__device__ __forceinline__ float max_chunk(const uint32_t (&s)[32], int nvalid, float acc)
+{
+    float m4[4] = {acc, -INFINITY, -INFINITY, -INFINITY};
+    #pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const float v = __uint_as_float(s[c]);
+        m4[c & 3] = fmaxf(m4[c & 3], (!kMasked || c < nvalid) ? v : -INFINITY);
+    }
+    return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+}
+
 template <int D>
 __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 2)
 block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
-                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_kc,
                          const __grid_constant__ CUtensorMap tm_v, const AttnArgs args)
 {
     using Cfg = AttnCfg<D>;
@@ -119,23 +168,20 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ---- set-up: barriers, TMEM, union of the two CSR rows
     if (tid == 0) {
         mbar_init(smem_u32(&ctl->q_full), 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&ctl->k_full[s]), 1);
-            mbar_init(smem_u32(&ctl->k_empty[s]), 1);
-            mbar_init(smem_u32(&ctl->v_full[s]), 1);
-            mbar_init(smem_u32(&ctl->v_empty[s]), 1);
-            mbar_init(smem_u32(&ctl->s_full[s]), 1);
-            mbar_init(smem_u32(&ctl->p_full[s]), 128);
-        }
-        mbar_init(smem_u32(&ctl->o_done), 1);
+        mbar_init(smem_u32(&ctl->k_full), 2);              // the two K producers arrive
+        mbar_init(smem_u32(&ctl->k_empty), 1);
+        mbar_init(smem_u32(&ctl->v_full), 1);
+        mbar_init(smem_u32(&ctl->v_empty), 1);
+        mbar_init(smem_u32(&ctl->s_full), 1);
+        mbar_init(smem_u32(&ctl->p_full), 128);
         mbar_init(smem_u32(&ctl->o_final), 1);
         mbar_init(smem_u32(&ctl->drain), 1);
         ctl->abort = 0;
         fence_mbar_init();
     }
-    if (warp == Cfg::PRODUCER_WARP && lane == 0) {
+    if (warp == Cfg::KA_WARP && lane == 0) {
         prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_kc);
         prefetch_tmap(&tm_v);
     }
     if (warp == 0) {
@@ -143,9 +189,8 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_relinquish();
     }
     // Union of the two CSR rows as bitmaps (one bit per key block and query
-    // block), built in the still unused K/V rings, then compacted in
-    // ascending order: a word's entries start at the popcount of all earlier
-    // words of (A | B).
+    // block), built in the still unused K stage, then compacted in ascending
+    // order: a word's entries start at the popcount of all earlier words.
     const int W = (Tb + 31) >> 5;                          // <= 128 words
     uint32_t* bmA = reinterpret_cast<uint32_t*>(base + Cfg::OFF_K);
     uint32_t* bmB = bmA + W;
@@ -174,7 +219,6 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     __syncthreads();
     if (warp == 0) {
-        // exclusive scan of per-word popcounts, 4 consecutive words per lane
         int cnt[4];
         int local = 0;
         #pragma unroll
@@ -201,170 +245,193 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncthreads();
     for (int w = tid; w < W; w += Cfg::THREADS) {
         const uint32_t a = bmA[w], b = bmB[w];
-        uint32_t u = a | b;
+        uint32_t m = a | b;
         int pos = word_off[w];
-        while (u) {
-            const int bit = __ffs(u) - 1;
-            u &= u - 1;
+        while (m) {
+            const int bit = __ffs(m) - 1;
+            m &= m - 1;
             list[pos++] = (w * 32 + bit) | (int32_t)(((a >> bit) & 1u) << 30) | (int32_t)(((b >> bit) & 1u) << 31);
         }
     }
     __syncthreads();
     const int L = ctl->list_len;
+    const int T = (L + 1) >> 1;                            // steps of two key blocks
     volatile int* abort = &ctl->abort;
 
-    if (warp == Cfg::PRODUCER_WARP) {
-        // ------------------------------------------------------------ TMA producer
+    // Key block of entry e (a missing second entry of the last step repeats
+    // the first one: valid data whose kept bits are 0).
+    auto block_of = [&](int e) -> int { return min((e < L ? list[e] : list[e - 1]) & 0x3fffffff, Tb - 1); };
+
+    if (warp == Cfg::KA_WARP || warp == Cfg::KB_WARP) {
+        // ------------------------------------------------ TMA: K of one key block per step
         if (lane == 0) {
-            fence_proxy_async_smem();   // the rings held the row bitmaps (generic accesses)
-            const uint32_t q_s = base_u32 + Cfg::OFF_Q;
-            mbar_arrive_expect_tx(smem_u32(&ctl->q_full), Cfg::Q_BYTES);
-            for (int c = 0; c < Cfg::KCH; ++c)
-                tma_load_3d(q_s + c * Cfg::Q_CHUNK, &tm_q, smem_u32(&ctl->q_full), c * 64, qb0 * 64, (int)bh);
-            int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
-            for (int t = 0; t < L; ++t) {
-                const int s = t % Cfg::STAGES;
-                const int use = t / Cfg::STAGES;
-                const int j = min(list[t] & 0x3fffffff, Tb - 1);
-                if (use > 0 && !mbar_wait(smem_u32(&ctl->k_empty[s]), (use - 1) & 1, abort, args.status)) break;
-                const uint32_t k_s = base_u32 + Cfg::OFF_K + s * Cfg::KV_BYTES;
-                mbar_arrive_expect_tx(smem_u32(&ctl->k_full[s]), Cfg::KV_BYTES);
-                for (int c = 0; c < Cfg::KCH; ++c)
-                    tma_load_3d(k_s + c * Cfg::KV_CHUNK, &tm_k, smem_u32(&ctl->k_full[s]), c * 64, j * 64, (int)bh);
-                issued_k[s] = use;
-                if (use > 0 && !mbar_wait(smem_u32(&ctl->v_empty[s]), (use - 1) & 1, abort, args.status)) break;
-                const uint32_t v_s = base_u32 + Cfg::OFF_V + s * Cfg::KV_BYTES;
-                mbar_arrive_expect_tx(smem_u32(&ctl->v_full[s]), Cfg::KV_BYTES);
-                for (int c = 0; c < Cfg::KCH; ++c)
-                    tma_load_3d(v_s + c * Cfg::KV_CHUNK, &tm_v, smem_u32(&ctl->v_full[s]), c * 64, j * 64, (int)bh);
-                issued_v[s] = use;
+            fence_proxy_async_smem();   // the stage held the row bitmaps (generic accesses)
+            const int g = (warp == Cfg::KA_WARP) ? 0 : 1;
+            int issued = -1;
+            if (g == 0) {
+                mbar_arrive_expect_tx(smem_u32(&ctl->q_full), Cfg::Q_BYTES);
+                tma_load_4d(base_u32 + Cfg::OFF_Q, &tm_q, smem_u32(&ctl->q_full), 0, qb0 * 64, 0, (int)bh);
             }
-            // Drain: no TMA may still be writing shared memory when the CTA
-            // exits.  Only this thread arms these barriers, so the phase of the
-            // last load it issued is the one to wait for.
-            mbar_wait_drain(smem_u32(&ctl->q_full), 0);
-            for (int s = 0; s < Cfg::STAGES; ++s) {
-                if (issued_k[s] >= 0) mbar_wait_drain(smem_u32(&ctl->k_full[s]), issued_k[s] & 1);
-                if (issued_v[s] >= 0) mbar_wait_drain(smem_u32(&ctl->v_full[s]), issued_v[s] & 1);
+            for (int t = 0; t < T; ++t) {
+                if (t > 0 && !mbar_wait(smem_u32(&ctl->k_empty), (t - 1) & 1, abort, args.status)) break;
+                const int j = block_of(2 * t + g);
+                const uint32_t dst = base_u32 + Cfg::OFF_K + g * 64 * 128;
+                mbar_arrive_expect_tx(smem_u32(&ctl->k_full), Cfg::KV_STAGE / 2);
+                for (int c = 0; c < Cfg::KCH; ++c)
+                    tma_load_3d(dst + c * Cfg::K_CHUNK, &tm_kc, smem_u32(&ctl->k_full), c * 64, j * 64, (int)bh);
+                issued = t;
             }
+            // Drain: no TMA may still be writing shared memory when the CTA exits.
+            if (g == 0) mbar_wait_drain(smem_u32(&ctl->q_full), 0);
+            if (issued >= 0) mbar_wait_drain(smem_u32(&ctl->k_full), issued & 1);
+        }
+    } else if (warp == Cfg::V_WARP) {
+        // ------------------------------------------------ TMA: V of both key blocks
+        if (lane == 0) {
+            fence_proxy_async_smem();
+            int issued = -1;
+            for (int t = 0; t < T; ++t) {
+                if (t > 0 && !mbar_wait(smem_u32(&ctl->v_empty), (t - 1) & 1, abort, args.status)) break;
+                const uint32_t dst = base_u32 + Cfg::OFF_V;
+                mbar_arrive_expect_tx(smem_u32(&ctl->v_full), Cfg::KV_STAGE);
+                for (int g = 0; g < 2; ++g)
+                    tma_load_4d(dst + g * Cfg::V_BLOCK, &tm_v, smem_u32(&ctl->v_full), 0, block_of(2 * t + g) * 64,
+                                0, (int)bh);
+                issued = t;
+            }
+            if (issued >= 0) mbar_wait_drain(smem_u32(&ctl->v_full), issued & 1);
         }
     } else if (warp == Cfg::MMA_WARP) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0);
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0);
             constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 1);
             const uint32_t q_s = base_u32 + Cfg::OFF_Q;
-            bool ok = (L == 0) || mbar_wait(smem_u32(&ctl->q_full), 0, abort, args.status);
+            const uint32_t k_s = base_u32 + Cfg::OFF_K;
+            const uint32_t v_s = base_u32 + Cfg::OFF_V;
+            bool ok = (T == 0) || mbar_wait(smem_u32(&ctl->q_full), 0, abort, args.status);
             tc_fence_after();
-            for (int t = 0; ok && t <= L; ++t) {
-                if (t < L) {
-                    const int s = t % Cfg::STAGES;
-                    if (!mbar_wait(smem_u32(&ctl->k_full[s]), (t / Cfg::STAGES) & 1, abort, args.status)) break;
-                    tc_fence_after();
-                    const uint32_t k_s = base_u32 + Cfg::OFF_K + s * Cfg::KV_BYTES;
-                    const uint32_t d_tmem = tmem + Cfg::TM_S + 64 * (t & 1);
-                    #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk & 3) * 32;   // 16 bf16 = 32 bytes per K step
-                        const uint64_t a = smem_desc_sw128(q_s + (kk >> 2) * Cfg::Q_CHUNK + off, 16, 1024);
-                        const uint64_t b = smem_desc_sw128(k_s + (kk >> 2) * Cfg::KV_CHUNK + off, 16, 1024);
-                        mma_ss(d_tmem, a, b, IDESC_S, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(smem_u32(&ctl->s_full[t & 1]));
-                    mma_commit(smem_u32(&ctl->k_empty[s]));
+            for (int t = 0; ok && t < T; ++t) {
+                const uint32_t par = t & 1;
+                if (!mbar_wait(smem_u32(&ctl->k_full), par, abort, args.status)) break;
+                tc_fence_after();
+                #pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk & 3) * 32;          // 16 bf16 = 32 bytes per K step
+                    const uint64_t a = smem_desc_sw128(q_s + (kk >> 2) * Cfg::Q_CHUNK + off, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(k_s + (kk >> 2) * Cfg::K_CHUNK + off, 16, 1024);
+                    mma_ss(tmem + Cfg::TM_S, a, b, IDESC_S, kk > 0 ? 1u : 0u);
                 }
-                if (t >= 1) {
-                    const int v = t - 1;
-                    const int s = v % Cfg::STAGES;
-                    if (!mbar_wait(smem_u32(&ctl->p_full[v & 1]), (v >> 1) & 1, abort, args.status)) break;
-                    if (!mbar_wait(smem_u32(&ctl->v_full[s]), (v / Cfg::STAGES) & 1, abort, args.status)) break;
-                    tc_fence_after();
-                    const uint32_t v_s = base_u32 + Cfg::OFF_V + s * Cfg::KV_BYTES;
-                    const uint32_t p_tmem = tmem + Cfg::TM_S + 64 * (v & 1);
-                    #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t b = smem_desc_sw128(v_s + kk * 2048, Cfg::KV_CHUNK, 1024);
-                        mma_ts(tmem + Cfg::TM_O, p_tmem + kk * 8, b, IDESC_O, (v > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(smem_u32(&ctl->o_done));
-                    mma_commit(smem_u32(&ctl->v_empty[s]));
-                    if (v == L - 1) mma_commit(smem_u32(&ctl->o_final));
+                mma_commit(smem_u32(&ctl->s_full));
+                mma_commit(smem_u32(&ctl->k_empty));
+                if (!mbar_wait(smem_u32(&ctl->p_full), par, abort, args.status)) break;
+                if (!mbar_wait(smem_u32(&ctl->v_full), par, abort, args.status)) break;
+                tc_fence_after();
+                #pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    // 16 keys per K step: steps 0-3 in block a, 4-7 in block b
+                    const uint64_t b = smem_desc_sw128(v_s + (kk >> 2) * Cfg::V_BLOCK + (kk & 3) * 2048, 64 * 128, 1024);
+                    mma_ts(tmem + Cfg::TM_O, tmem + Cfg::TM_S + kk * 8, b, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
                 }
+                mma_commit(smem_u32(&ctl->v_empty));
+                if (t == T - 1) mma_commit(smem_u32(&ctl->o_final));
             }
             // Drain: every MMA this thread issued has completed before TMEM is freed.
             mma_commit(smem_u32(&ctl->drain));
             mbar_wait_drain(smem_u32(&ctl->drain), 0);
         }
     } else {
-        // ------------------------------------------------------------ softmax + epilogue
+        // ------------------------------------------------ softmax + epilogue (warps 0-3)
         const int row = tid;                       // 0..127 = TMEM lane
         const int half = row >> 6;                 // which query block of the pair
         const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+        const uint32_t s_row = tmem + lane_addr + Cfg::TM_S;
         const float sl2 = args.scale_log2;
         float m_run = -INFINITY;
         float l_run = 0.f;
         bool ok = true;
-        for (int t = 0; t < L; ++t) {
-            const int b = t & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl->s_full[b]), (t >> 1) & 1, abort, args.status));
+        for (int t = 0; t < T; ++t) {
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl->s_full), t & 1, abort, args.status));
             if (!ok) break;
             tc_fence_after();
-            const int32_t e = list[t];
-            const int j = e & 0x3fffffff;
-            const bool kept = (e >> (30 + half)) & 1;        // uniform over the warp
-            const uint32_t s_addr = tmem + lane_addr + Cfg::TM_S + 64 * b;
-            uint32_t pk[32];
-            if (kept) {
-                uint32_t sr[64];
-                tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_wait_ld();
-                const int nvalid = min(64, args.N - j * 64);
-                float smax = -INFINITY;
-                #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (c < nvalid) smax = fmaxf(smax, __uint_as_float(sr[c]));
-                const float mb = smax * sl2;                  // scale > 0: max commutes
-                const bool need = (m_run != -INFINITY) && (mb > m_run + 8.0f);
-                if (__any_sync(0xffffffffu, need)) {
-                    // O rescale: the PV product of step t-1 must be complete (t >= 1 here).
-                    float f = 1.f;
-                    if (need) { f = ex2_approx(m_run - mb); l_run *= f; m_run = mb; }
-                    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl->o_done), (t - 1) & 1, abort, args.status));
-                    if (!ok) break;
-                    tc_fence_after();
-                    #pragma unroll 1
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_addr + Cfg::TM_O + c0, o);
-                        tmem_wait_ld();
-                        #pragma unroll
-                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-                        tmem_st32(tmem + lane_addr + Cfg::TM_O + c0, o);
-                    }
-                }
-                if (m_run == -INFINITY) m_run = mb;
-                const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
-                float sum = 0.f;
-                #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const float p0 = (c < nvalid) ? ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, neg_mu)) : 0.f;
-                    const float p1 = (c + 1 < nvalid) ? ex2_approx(fmaf(__uint_as_float(sr[c + 1]), sl2, neg_mu)) : 0.f;
-                    sum += p0 + p1;
-                    pk[c >> 1] = pack_bf16x2(p0, p1);
-                }
-                l_run += sum;
-            } else {
-                #pragma unroll
-                for (int c = 0; c < 32; ++c) pk[c] = 0u;
+            // kept flags and valid key counts of the step's two key blocks (uniform over the warp)
+            bool kept[2];
+            int nv[2];
+            #pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                const int e = 2 * t + g;
+                const int32_t ent = (e < L) ? list[e] : 0;
+                kept[g] = (e < L) && ((ent >> (30 + half)) & 1);
+                nv[g] = min(64, args.N - (ent & 0x3fffffff) * 64);
             }
-            tmem_st32(s_addr, pk);
+            // pass 1: row max over the kept blocks
+            float mx = -INFINITY;
+            #pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                if (!kept[g]) continue;
+                uint32_t a[32], b[32];
+                tmem_ld32(s_row + 64 * g, a);
+                tmem_ld32(s_row + 64 * g + 32, b);
+                tmem_wait_ld();
+                if (nv[g] == 64) {
+                    mx = max_chunk<false>(a, 64, mx);
+                    mx = max_chunk<false>(b, 64, mx);
+                } else {
+                    mx = max_chunk<true>(a, nv[g], mx);
+                    mx = max_chunk<true>(b, nv[g] - 32, mx);
+                }
+            }
+            const float mb = mx * sl2;                     // scale > 0: max commutes
+            const bool need = (m_run != -INFINITY) && (mb > m_run + 8.0f);
+            if (__any_sync(0xffffffffu, need)) {
+                // Rescale O: PV_{t-1} was issued before S_t, so it is complete.
+                float f = 1.f;
+                if (need) { f = ex2_approx(m_run - mb); l_run *= f; m_run = mb; }
+                #pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_addr + Cfg::TM_O + c0, o);
+                    tmem_wait_ld();
+                    #pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+                    tmem_st32(tmem + lane_addr + Cfg::TM_O + c0, o);
+                }
+            }
+            if (m_run == -INFINITY) m_run = mb;
+            const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
+            // pass 2: P = 2^(s*sl2 - m) in bf16 over the first 64 columns of S,
+            // chunk q of 32 scores -> 16 columns at 16q (behind every chunk read)
+            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+            #pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                uint32_t pk[16];
+                if (kept[g]) {
+                    uint32_t a[32];
+                    tmem_ld32(s_row + 64 * g, a);
+                    tmem_wait_ld();
+                    uint32_t b[32];
+                    tmem_ld32(s_row + 64 * g + 32, b);         // in flight during the first half
+                    if (nv[g] == 64) exp_chunk<false>(a, sl2, neg_mu, 32, pk, sum4);
+                    else exp_chunk<true>(a, sl2, neg_mu, nv[g], pk, sum4);
+                    tmem_st16(s_row + 32 * g, pk);
+                    tmem_wait_ld();
+                    if (nv[g] == 64) exp_chunk<false>(b, sl2, neg_mu, 32, pk, sum4);
+                    else exp_chunk<true>(b, sl2, neg_mu, nv[g] - 32, pk, sum4);
+                    tmem_st16(s_row + 32 * g + 16, pk);
+                } else {
+                    #pragma unroll
+                    for (int c = 0; c < 16; ++c) pk[c] = 0u;
+                    tmem_st16(s_row + 32 * g, pk);
+                    tmem_st16(s_row + 32 * g + 16, pk);
+                }
+            }
+            l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(smem_u32(&ctl->p_full[b]));
+            mbar_arrive(smem_u32(&ctl->p_full));
         }
         // ---- epilogue: O / l -> bf16
-        if (ok && L > 0)
+        if (ok && T > 0)
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl->o_final), 0, abort, args.status));
         tc_fence_after();
         if (ok) {
@@ -376,7 +443,7 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             #pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t o[32];
-                if (L > 0) {
+                if (T > 0) {
                     tmem_ld32(tmem + lane_addr + Cfg::TM_O + c0, o);
                     tmem_wait_ld();
                 } else {

@@ -91,10 +91,27 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity)
     return true;
 }
 
+// Barrier among `nthreads` threads (a multiple of 32) of the CTA, id 1..15.
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // -------------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// 4D tiled load into this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
+                                            int32_t x, int32_t y, int32_t z, int32_t w)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
 }
 
 // 3D tiled load into this CTA's shared memory, completing on `bar`.
@@ -196,6 +213,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+          "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 // Shared-memory matrix descriptor (sm_100 layout): start address, leading and
 // stride byte offsets (16-byte units), descriptor version 1, 128-byte swizzle.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes)
@@ -226,6 +254,24 @@ __device__ __forceinline__ float ex2_approx(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA pipe, for softmax arguments (x <= 8): x = j + f with j the
+// nearest integer (adding 1.5*2^23 rounds x into the low mantissa bits) and
+// f in [-0.5, 0.5]; 2^f from a cubic fitted for least maximum relative error
+// on that interval (max rel. error 7.5e-5, well below bf16's 2^-9 half-ulp);
+// 2^j by adding j to the exponent field.  Arguments below -125 are clamped
+// (the result is then ~2^-125, nothing at bf16 / fp32-sum precision).
+__device__ __forceinline__ float exp2_poly(float x)
+{
+    x = fmaxf(x, -125.f);
+    const float kRound = 12582912.f;
+    const float t = x + kRound;
+    const float f = x - (t - kRound);
+    float p = fmaf(0.0551716685295105f, f, 0.2426111400127411f);
+    p = fmaf(p, f, 0.6932609677314758f);
+    p = fmaf(p, f, 0.9999280571937561f);
+    return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - __float_as_int(kRound)) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)

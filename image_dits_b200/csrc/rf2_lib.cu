@@ -169,6 +169,24 @@ static bool make_map(CUtensorMap* m, const void* ptr, int32_t D, int32_t N, int6
     return r == CUDA_SUCCESS;
 }
 
+// The same tensor viewed as 4D (64 columns, N rows, D/64 column chunks, BH):
+// one box = `box_rows` rows x all of d, landing in shared memory chunk by
+// chunk ([chunk][row][64 columns], 128-byte swizzle), i.e. one TMA load per
+// tile instead of one per 64-column chunk.
+static bool make_map_chunked(CUtensorMap* m, const void* ptr, int32_t D, int32_t N, int64_t BH, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {64, (cuuint64_t)N, (cuuint64_t)(D / 64), (cuuint64_t)BH};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, 128, (cuuint64_t)N * D * 2};
+    const cuuint32_t box[4] = {64, box_rows, (cuuint32_t)(D / 64), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 static int* status_word_ptr()
 {
     int* p = nullptr;
@@ -183,8 +201,8 @@ static int launch_attn(const Checked& c, const MaskGeo& mg, const void* qp, cons
 {
     using Cfg = AttnCfg<D>;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, qp, D, c.N, c.BH, 128) || !make_map(&mk, kp, D, c.N, c.BH, 64) ||
-        !make_map(&mv, vp, D, c.N, c.BH, 64))
+    if (!make_map_chunked(&mq, qp, D, c.N, c.BH, 128) || !make_map(&mk, kp, D, c.N, c.BH, 64) ||
+        !make_map_chunked(&mv, vp, D, c.N, c.BH, 64))
         return RF2_ERR_CUDA;
     int* status = status_word_ptr();
     if (!status) return RF2_ERR_CUDA;
