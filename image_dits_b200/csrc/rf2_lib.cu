@@ -106,9 +106,9 @@ static int grid_for_rows(int64_t rows)
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t warps = (rows + 31) / 32;
+    const int64_t warps = (rows + RF2_PERMUTE_ROWS - 1) / RF2_PERMUTE_ROWS;
     int64_t blocks = (warps + 7) / 8;
-    const int64_t cap = (int64_t)sms * 8;
+    const int64_t cap = (int64_t)sms * RF2_PERMUTE_MINB * 4;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     return (int)blocks;
