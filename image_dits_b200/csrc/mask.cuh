@@ -6,15 +6,19 @@
 //                     the permuted tensors, so this is a segmented reduction
 //                     over contiguous memory: one warp per block, 16-byte
 //                     loads, fp32 accumulation, HBM-bound.
-// select_kernel       S^_ij = q^_i . k^_j / sqrt(d) for R query blocks of one
-//                     head against every key block (fp32 FMA from shared
-//                     memory, eq. (7)), then per row the n largest scores
-//                     (eq. (8)) by a 4-pass 8-bit radix select on
-//                     order-preserving uint32 keys (equal scores: lower j),
-//                     union the sink columns, and write the row as an
-//                     ascending CSR list.  Sink rows keep every column.
+// score_tc_kernel     S^_ij = q^_i . k^_j / sqrt(d) (eq. (7)) for a group of
+//                     heads on the tensor cores (tcgen05 kind::tf32, three
+//                     hi/lo products for fp32 accuracy), into a score buffer
+//                     that stays in L2 between the two kernels.
+// select_from_scores_kernel
+//                     per row the n largest scores (eq. (8)) by a 4-pass
+//                     8-bit radix select on order-preserving uint32 keys
+//                     (equal scores: lower j), union the sink columns, and
+//                     write the row as an ascending CSR list.  Sink rows keep
+//                     every column.
 #pragma once
 #include "geometry.cuh"
+#include "ptx.cuh"
 
 namespace rf2 {
 
@@ -28,12 +32,14 @@ __device__ __forceinline__ void bf16x8_accumulate(const uint4 v, float (&acc)[8]
     }
 }
 
-// means: [2][BH][Tb][D] fp32 (0 = queries, 1 = keys).
+// Output: the block means as a tf32 split, hi = tf32(mean) (low 13 mantissa
+// bits zero) and lo = mean - hi, each [2][BH][Tb][D] fp32 (0 = queries,
+// 1 = keys), ready for the tensor-core score kernel.
 template <int D>
 __global__ void __launch_bounds__(256) block_mean_kernel(const uint4* __restrict__ qp,
                                                          const uint4* __restrict__ kp,
-                                                         float* __restrict__ means, int32_t N,
-                                                         int32_t Tb, int64_t BH)
+                                                         float* __restrict__ means_hi, float* __restrict__ means_lo,
+                                                         int32_t N, int32_t Tb, int64_t BH)
 {
     constexpr int C = D / 8;
     constexpr int R = 32 / C;
@@ -65,9 +71,16 @@ __global__ void __launch_bounds__(256) block_mean_kernel(const uint4* __restrict
         for (int k = 0; k < 8; ++k) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], off);
     if (lane < C) {
         const float fr = (float)rows;
-        float4* dst = reinterpret_cast<float4*>(means + ((int64_t)which * per_tensor + rem) * D) + 2 * cidx;
-        dst[0] = make_float4(acc[0] / fr, acc[1] / fr, acc[2] / fr, acc[3] / fr);
-        dst[1] = make_float4(acc[4] / fr, acc[5] / fr, acc[6] / fr, acc[7] / fr);
+        const int64_t at = ((int64_t)which * per_tensor + rem) * D + 8 * cidx;
+        float m[8], h[8];
+        #pragma unroll
+        for (int k = 0; k < 8; ++k) { m[k] = acc[k] / fr; h[k] = to_tf32(m[k]); }
+        float4* dh = reinterpret_cast<float4*>(means_hi + at);
+        float4* dl = reinterpret_cast<float4*>(means_lo + at);
+        dh[0] = make_float4(h[0], h[1], h[2], h[3]);
+        dh[1] = make_float4(h[4], h[5], h[6], h[7]);
+        dl[0] = make_float4(m[0] - h[0], m[1] - h[1], m[2] - h[2], m[3] - h[3]);
+        dl[1] = make_float4(m[4] - h[4], m[5] - h[5], m[6] - h[6], m[7] - h[7]);
     }
 }
 
@@ -79,171 +92,331 @@ __device__ __forceinline__ uint32_t float_order_key(float f)
 }
 
 constexpr int kSelThreads = 256;
-constexpr int kSelKeysPerChunk = 64;
 
-template <int D, int R>
-struct SelectSmem {
-    static constexpr int KSTRIDE = D + 4;       // padded row of a key-mean chunk (floats)
-    static size_t bytes(int Tb)
-    {
-        return sizeof(float) * (size_t)R * D                                  // query means
-             + sizeof(float) * (size_t)kSelKeysPerChunk * KSTRIDE             // key-mean chunk
-             + sizeof(uint32_t) * (size_t)R * Tb                              // score keys
-             + sizeof(uint32_t) * 256 * (kSelThreads / 32);                   // histograms
+// Selection of one non-sink or sink row i of head bh from its T_b score keys
+// (order-preserving uint32), by one warp: the n-th largest key by a 4-pass
+// 8-bit radix select (hist: 256 words of this warp's shared memory), then the
+// kept set {key > thr} + the lowest-indexed keys == thr up to n, plus every
+// sink column, written in ascending order at the row's closed-form offset.
+__device__ __forceinline__ void select_row(const uint32_t* rk, uint32_t* hist, const MaskGeo& mg, int64_t bh, int i,
+                                           int lane, int32_t* row_start, int32_t* row_count, int32_t* col_idx,
+                                           bool keep_all)
+{
+    const int Tb = mg.Tb;
+    const int64_t rs = row_offset(mg, bh, i);
+    const int64_t row_id = bh * Tb + i;
+    int32_t* out = col_idx + rs;
+    if (i >= mg.sink_first || keep_all) {
+        for (int j = lane; j < Tb; j += 32) out[j] = j;
+        if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = Tb; }
+        return;
     }
+    // Keys of a row often share many leading bits (scores cluster): start the
+    // 8-bit digits just below the bits common to the row's min and max key.
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int j = lane; j < Tb; j += 32) { const uint32_t k = rk[j]; kmin = min(kmin, k); kmax = max(kmax, k); }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const int common = __clz(kmin ^ kmax);                  // 32 when every key is equal
+    uint32_t pmask = (common >= 32) ? 0xffffffffu : ~(0xffffffffu >> common);
+    uint32_t prefix = kmax & pmask;
+    int remaining = mg.n_keep;
+    const int top = 32 - common;                            // undetermined low bits
+    #pragma unroll 1
+    for (int lo = top - 8; lo > -8; lo -= 8) {
+        const int shift = (lo < 0) ? 0 : lo;                // the last digit may overlap fixed bits
+
+        #pragma unroll
+        for (int b = 0; b < 8; ++b) hist[lane * 8 + b] = 0;
+        __syncwarp();
+        // Lanes hitting the same bin add once (the scores of a row are
+        // concentrated, so a warp's 32 keys often share one or two bins).
+        for (int j0 = 0; j0 < Tb; j0 += 32) {
+            const int j = j0 + lane;
+            const uint32_t k = (j < Tb) ? rk[j] : 0u;
+            const bool hit = (j < Tb) && ((k & pmask) == prefix);
+            const uint32_t bin = hit ? ((k >> shift) & 255u) : 256u;
+            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+            if (hit && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+        }
+        __syncwarp();
+        // Lane l owns bins 255-8l .. 248-8l (descending).
+        uint32_t cnt[8];
+        uint32_t local = 0;
+        #pragma unroll
+        for (int b = 0; b < 8; ++b) { cnt[b] = hist[255 - (lane * 8 + b)]; local += cnt[b]; }
+        uint32_t incl = local;
+        #pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        const uint32_t excl = incl - local;
+        const bool here = (excl < (uint32_t)remaining) && ((uint32_t)remaining <= incl);
+        const uint32_t ballot = __ballot_sync(0xffffffffu, here);
+        const int src_lane = __ffs(ballot) - 1;
+        uint32_t bin = 0, before = 0;
+        if (lane == src_lane) {
+            uint32_t run = excl;
+            #pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                if (run + cnt[b] >= (uint32_t)remaining) { bin = 255 - (lane * 8 + b); before = run; break; }
+                run += cnt[b];
+            }
+        }
+        bin = __shfl_sync(0xffffffffu, bin, src_lane);
+        before = __shfl_sync(0xffffffffu, before, src_lane);
+        remaining -= (int)before;
+        prefix |= bin << shift;
+        pmask |= 255u << shift;
+        __syncwarp();
+    }
+    // prefix is the threshold key; `remaining` keys equal to it are kept,
+    // the lowest-indexed ones first.
+    const uint32_t thr = prefix;
+    int eq_left = remaining;
+    int written = 0;
+    for (int j0 = 0; j0 < Tb; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t k = (j < Tb) ? rk[j] : 0u;
+        const bool eq = (j < Tb) && (k == thr);
+        const uint32_t eq_ballot = __ballot_sync(0xffffffffu, eq);
+        const int eq_rank = __popc(eq_ballot & ((1u << lane) - 1u));
+        const bool sel = (j < Tb) && (k > thr || (eq && eq_rank < eq_left) || j >= mg.sink_first);
+        eq_left -= __popc(eq_ballot);
+        const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[written + __popc(sel_ballot & ((1u << lane) - 1u))] = j;
+        written += __popc(sel_ballot);
+    }
+    if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = written; }
+}
+
+// ------------------------------------------------------------------------
+// Pooled scores on the tensor cores (eq. (7)): S^ = q^ k^T / sqrt(d) for a
+// group of heads, as tcgen05 kind::tf32 products of the hi/lo split written
+// by block_mean_kernel: q.k = hi.hi + hi.lo + lo.hi, leaving about 2^-21
+// |q||k| of error, far inside the 1e-5 tie band of the selection.
+// Work item = (head, 128 query blocks); persistent CTAs take items i,
+// i + gridDim.x, ...  An item walks its key blocks in chunks of 256 (one
+// M128 x N256 accumulator) and d in slices of 32; each stage holds the query
+// slice (hi, lo) and the key slice (hi, lo).
+// Roles (256 threads): warps 0 and 1 issue the TMA loads (hi and lo parts:
+// one thread's TMA stream is served serially); warp 2 issues the MMAs into
+// one of two 256-column TMEM accumulators; warps 4-7 move a finished
+// accumulator to S^ in global memory, scaled by 1/sqrt(d), while the next
+// chunk is multiplied.
+template <int D>
+struct ScoreCfg {
+    static constexpr int KC = D / 32;                  // 32-float (128-byte) slices of d
+    static constexpr int NCH = 256;                    // keys per accumulator
+    static constexpr uint32_t A_TILE = 128 * 128;      // 128 rows x 32 floats
+    static constexpr uint32_t B_TILE = NCH * 128;      // 256 rows x 32 floats
+    static constexpr uint32_t STAGE = 2 * A_TILE + 2 * B_TILE;   // [A hi][A lo][B hi][B lo]
+    static constexpr uint32_t SMEM = 1024 + 2 * STAGE + 128;
+    static constexpr int THREADS = 256;
 };
 
-// Grid: (ceil(Tb / R), BH).  Block: 256 threads.
-template <int D, int R>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ means,
-                                                             int32_t* __restrict__ row_start,
-                                                             int32_t* __restrict__ row_count,
-                                                             int32_t* __restrict__ col_idx,
-                                                             MaskGeo mg, int64_t BH, float inv_sqrt_d)
+template <int D>
+__global__ void __launch_bounds__(ScoreCfg<D>::THREADS, 1)
+score_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
+                const __grid_constant__ CUtensorMap tm_hi_b, const __grid_constant__ CUtensorMap tm_lo_b,
+                float* __restrict__ S, int32_t Tb, int32_t ld_s, int64_t BH, int64_t h0, int32_t G,
+                float inv_sqrt_d, int* status)
 {
-    using SM = SelectSmem<D, R>;
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    float* qs = reinterpret_cast<float*>(smem_raw);                       // [R][D]
-    float* ks = qs + R * D;                                               // [64][D+4]
-    uint32_t* keys = reinterpret_cast<uint32_t*>(ks + kSelKeysPerChunk * SM::KSTRIDE);  // [R][Tb]
-    uint32_t* hist_all = keys + (size_t)R * mg.Tb;                        // [8][256]
+    using Cfg = ScoreCfg<D>;
+    constexpr int KC = Cfg::KC;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+    uint8_t* base = smem_raw + (base_u32 - raw_u32);
+    // barriers: full[2], empty[2], acc_full[2], acc_empty[2], drain
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + 2 * Cfg::STAGE);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + 2;
+    uint64_t* acc_full = bars + 4;
+    uint64_t* acc_empty = bars + 6;
+    uint64_t* drain = bars + 8;
 
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int mtiles = (Tb + 127) / 128;
+    const int nchunks = (Tb + Cfg::NCH - 1) / Cfg::NCH;
+    const int items = G * mtiles;
+    const int my_items = (blockIdx.x < items) ? (items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&full[i]), 2);                 // hi and lo producers
+            mbar_init(smem_u32(&empty[i]), 1);
+            mbar_init(smem_u32(&acc_full[i]), 1);
+            mbar_init(smem_u32(&acc_empty[i]), 128);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    volatile int* abort = abort_flag;
+
+    if (warp == 0 || warp == 1) {
+        if (lane == 0) {
+            // warp 0: hi parts, warp 1: lo parts.  Rows of the block-mean maps:
+            // queries of all heads first, then keys.
+            const CUtensorMap* ta = (warp == 0) ? &tm_hi : &tm_lo;
+            const CUtensorMap* tb = (warp == 0) ? &tm_hi_b : &tm_lo_b;
+            int step = 0;
+            int issued[2] = {-1, -1};
+            bool ok = true;
+            for (int it = 0; ok && it < my_items; ++it) {
+                const int item = blockIdx.x + it * gridDim.x;
+                const int64_t bh = h0 + item / mtiles;
+                const int m0 = (item % mtiles) * 128;
+                const int qrow = (int)(bh * Tb) + m0;
+                const int krow0 = (int)(BH * Tb + bh * Tb);
+                for (int n = 0; ok && n < nchunks; ++n)
+                    for (int c = 0; c < KC; ++c, ++step) {
+                        const int b = step & 1;
+                        const int use = step >> 1;
+                        if (use > 0 && !mbar_wait(smem_u32(&empty[b]), (use - 1) & 1, abort, status)) { ok = false; break; }
+                        const uint32_t st = base_u32 + b * Cfg::STAGE;
+                        mbar_arrive_expect_tx(smem_u32(&full[b]), Cfg::A_TILE + Cfg::B_TILE);
+                        tma_load_2d(st + warp * Cfg::A_TILE, ta, smem_u32(&full[b]), c * 32, qrow);
+                        tma_load_2d(st + 2 * Cfg::A_TILE + warp * Cfg::B_TILE, tb, smem_u32(&full[b]), c * 32,
+                                    krow0 + n * Cfg::NCH);
+                        issued[b] = use;
+                    }
+            }
+            for (int b = 0; b < 2; ++b)
+                if (issued[b] >= 0) mbar_wait_drain(smem_u32(&full[b]), issued[b] & 1);
+        }
+    } else if (warp == 2) {
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_tf32_f32(128, Cfg::NCH);
+            int step = 0, chunk = 0;
+            bool ok = true;
+            for (int it = 0; ok && it < my_items; ++it)
+                for (int n = 0; ok && n < nchunks; ++n, ++chunk) {
+                    const int a = chunk & 1;
+                    if (chunk >= 2 && !mbar_wait(smem_u32(&acc_empty[a]), ((chunk >> 1) - 1) & 1, abort, status)) { ok = false; break; }
+                    const uint32_t d_tmem = tmem + Cfg::NCH * a;
+                    for (int c = 0; c < KC; ++c, ++step) {
+                        const int b = step & 1;
+                        if (!mbar_wait(smem_u32(&full[b]), (step >> 1) & 1, abort, status)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t st = base_u32 + b * Cfg::STAGE;
+                        const uint32_t a_hi = st, a_lo = st + Cfg::A_TILE;
+                        const uint32_t b_hi = st + 2 * Cfg::A_TILE, b_lo = b_hi + Cfg::B_TILE;
+                        #pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {              // 8 floats = 32 bytes per K step
+                            const uint32_t off = ks * 32;
+                            const uint32_t first = (c == 0 && ks == 0) ? 0u : 1u;
+                            mma_ss_tf32(d_tmem, smem_desc_sw128(a_hi + off, 16, 1024), smem_desc_sw128(b_hi + off, 16, 1024), IDESC, first);
+                            mma_ss_tf32(d_tmem, smem_desc_sw128(a_hi + off, 16, 1024), smem_desc_sw128(b_lo + off, 16, 1024), IDESC, 1u);
+                            mma_ss_tf32(d_tmem, smem_desc_sw128(a_lo + off, 16, 1024), smem_desc_sw128(b_hi + off, 16, 1024), IDESC, 1u);
+                        }
+                        mma_commit(smem_u32(&empty[b]));
+                    }
+                    if (ok) mma_commit(smem_u32(&acc_full[a]));
+                }
+            mma_commit(smem_u32(drain));
+            mbar_wait_drain(smem_u32(drain), 0);
+        }
+    } else if (warp >= 4) {
+        // epilogue warps 4-7: TMEM lane quarter = warp % 4, so row = 32 * (warp % 4) + lane
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        bool ok = true;
+        int chunk = 0;
+        for (int it = 0; ok && it < my_items; ++it) {
+            const int item = blockIdx.x + it * gridDim.x;
+            const int64_t hl = item / mtiles;                  // head within the group
+            const int i = (item % mtiles) * 128 + row;
+            float* dst = S + (hl * Tb + i) * (int64_t)ld_s;
+            for (int n = 0; n < nchunks; ++n, ++chunk) {
+                const int a = chunk & 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[a]), (chunk >> 1) & 1, abort, status));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t taddr = tmem + lane_addr + Cfg::NCH * a;
+                #pragma unroll 1
+                for (int c0 = 0; c0 < Cfg::NCH; c0 += 32) {
+                    const int j0 = n * Cfg::NCH + c0;
+                    if (j0 >= Tb) break;                        // uniform over the warp
+                    uint32_t r[32];
+                    tmem_ld32(taddr + c0, r);
+                    tmem_wait_ld();
+                    if (i < Tb) {
+                        if (j0 + 32 <= Tb) {
+                            #pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                reinterpret_cast<float4*>(dst + j0)[q] = make_float4(
+                                    __uint_as_float(r[4 * q]) * inv_sqrt_d, __uint_as_float(r[4 * q + 1]) * inv_sqrt_d,
+                                    __uint_as_float(r[4 * q + 2]) * inv_sqrt_d, __uint_as_float(r[4 * q + 3]) * inv_sqrt_d);
+                        } else {
+                            #pragma unroll
+                            for (int q = 0; q < 32; ++q)
+                                if (j0 + q < Tb) dst[j0 + q] = __uint_as_float(r[q]) * inv_sqrt_d;
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&acc_empty[a]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------------
+// Top-n per row + sink + CSR (eq. (8), section 3.4) from precomputed scores:
+// R rows of one head per CTA (256 threads), the rows' scores loaded as
+// order-preserving keys into shared memory, then one warp per row: 4-pass
+// 8-bit radix select of the n-th largest key (equal scores: lower j), and an
+// ascending ballot-ordered CSR write including every sink column.
+template <int R>
+__global__ void __launch_bounds__(kSelThreads) select_from_scores_kernel(const float* __restrict__ S, int32_t ld_s,
+                                                                         int32_t* __restrict__ row_start,
+                                                                         int32_t* __restrict__ row_count,
+                                                                         int32_t* __restrict__ col_idx, MaskGeo mg,
+                                                                         int64_t h0)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
     const int Tb = mg.Tb;
-    const int64_t bh = blockIdx.y;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw);            // [R][Tb]
+    uint32_t* hist_all = keys + (size_t)R * Tb;                          // [8][256]
+    const int64_t hl = blockIdx.y;                                        // head within the group
+    const int64_t bh = h0 + hl;
     const int i0 = blockIdx.x * R;
     const int nrows = min(R, Tb - i0);
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
-    const float* qm = means + (bh * Tb) * D;
-    const float* km = means + (BH * Tb + bh * Tb) * D;
-
-    // Rows of this tile that need scoring (sink rows keep every column).
-    const int n_score_rows = max(0, min(nrows, mg.sink_first - i0));
     const bool keep_all = mg.n_keep >= Tb;
-
-    if (n_score_rows > 0 && !keep_all) {
-        for (int e = tid; e < R * D / 4; e += kSelThreads) {
-            const int r = (e * 4) / D;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r < n_score_rows) v = reinterpret_cast<const float4*>(qm + (int64_t)i0 * D)[e];
-            reinterpret_cast<float4*>(qs)[e] = v;
-        }
-        // Thread layout for scoring: key kk = tid % 64, rows rg*(R/4) .. +R/4.
-        constexpr int RPT = R / 4;
-        const int kk = tid % kSelKeysPerChunk;
-        const int rg = tid / kSelKeysPerChunk;
-        for (int j0 = 0; j0 < Tb; j0 += kSelKeysPerChunk) {
-            __syncthreads();
-            const int nk = min(kSelKeysPerChunk, Tb - j0);
-            for (int e = tid; e < kSelKeysPerChunk * D / 4; e += kSelThreads) {
-                const int kr = (e * 4) / D;
-                const int kc = (e * 4) % D;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (kr < nk) v = reinterpret_cast<const float4*>(km + (int64_t)(j0 + kr) * D)[kc / 4];
-                *reinterpret_cast<float4*>(ks + kr * SM::KSTRIDE + kc) = v;
-            }
-            __syncthreads();
-            float acc[RPT];
-            #pragma unroll
-            for (int r = 0; r < RPT; ++r) acc[r] = 0.f;
-            const float* krow = ks + kk * SM::KSTRIDE;
-            #pragma unroll 4
-            for (int c = 0; c < D; c += 4) {
-                const float4 kv = *reinterpret_cast<const float4*>(krow + c);
-                #pragma unroll
-                for (int r = 0; r < RPT; ++r) {
-                    const float4 qv = *reinterpret_cast<const float4*>(qs + (rg * RPT + r) * D + c);
-                    acc[r] = fmaf(qv.x, kv.x, acc[r]);
-                    acc[r] = fmaf(qv.y, kv.y, acc[r]);
-                    acc[r] = fmaf(qv.z, kv.z, acc[r]);
-                    acc[r] = fmaf(qv.w, kv.w, acc[r]);
-                }
-            }
-            if (kk < nk) {
-                #pragma unroll
-                for (int r = 0; r < RPT; ++r)
-                    keys[(size_t)(rg * RPT + r) * Tb + j0 + kk] = float_order_key(acc[r] * inv_sqrt_d);
-            }
-        }
-        __syncthreads();
+    const int n_score_rows = keep_all ? 0 : max(0, min(nrows, mg.sink_first - i0));
+    for (int r = 0; r < n_score_rows; ++r) {
+        const float* src = S + (hl * Tb + i0 + r) * (int64_t)ld_s;
+        for (int j = tid; j < Tb; j += kSelThreads) keys[(size_t)r * Tb + j] = float_order_key(src[j]);
     }
-
+    __syncthreads();
     uint32_t* hist = hist_all + warp * 256;
-    for (int r = warp; r < nrows; r += kSelThreads / 32) {
-        const int i = i0 + r;
-        const int64_t rs = row_offset(mg, bh, i);
-        const int64_t row_id = bh * Tb + i;
-        int32_t* out = col_idx + rs;
-        if (i >= mg.sink_first || keep_all) {
-            for (int j = lane; j < Tb; j += 32) out[j] = j;
-            if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = Tb; }
-            continue;
-        }
-        const uint32_t* rk = keys + (size_t)r * Tb;
-        // Radix select of the n-th largest key, 8 bits at a time from the top.
-        uint32_t prefix = 0, pmask = 0;
-        int remaining = mg.n_keep;
-        #pragma unroll 1
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            #pragma unroll
-            for (int b = 0; b < 8; ++b) hist[lane * 8 + b] = 0;
-            __syncwarp();
-            for (int j = lane; j < Tb; j += 32) {
-                const uint32_t k = rk[j];
-                if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
-            }
-            __syncwarp();
-            // Lane l owns bins 255-8l .. 248-8l (descending).
-            uint32_t cnt[8];
-            uint32_t local = 0;
-            #pragma unroll
-            for (int b = 0; b < 8; ++b) { cnt[b] = hist[255 - (lane * 8 + b)]; local += cnt[b]; }
-            uint32_t incl = local;
-            #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += v;
-            }
-            const uint32_t excl = incl - local;
-            const bool here = (excl < (uint32_t)remaining) && ((uint32_t)remaining <= incl);
-            const uint32_t ballot = __ballot_sync(0xffffffffu, here);
-            const int src_lane = __ffs(ballot) - 1;
-            uint32_t bin = 0, before = 0;
-            if (lane == src_lane) {
-                uint32_t run = excl;
-                #pragma unroll
-                for (int b = 0; b < 8; ++b) {
-                    if (run + cnt[b] >= (uint32_t)remaining) { bin = 255 - (lane * 8 + b); before = run; break; }
-                    run += cnt[b];
-                }
-            }
-            bin = __shfl_sync(0xffffffffu, bin, src_lane);
-            before = __shfl_sync(0xffffffffu, before, src_lane);
-            remaining -= (int)before;
-            prefix |= bin << shift;
-            pmask |= 255u << shift;
-            __syncwarp();
-        }
-        // prefix is the threshold key; `remaining` keys equal to it are kept,
-        // the lowest-indexed ones first.
-        const uint32_t thr = prefix;
-        int eq_left = remaining;
-        int written = 0;
-        for (int j0 = 0; j0 < Tb; j0 += 32) {
-            const int j = j0 + lane;
-            const uint32_t k = (j < Tb) ? rk[j] : 0u;
-            const bool eq = (j < Tb) && (k == thr);
-            const uint32_t eq_ballot = __ballot_sync(0xffffffffu, eq);
-            const int eq_rank = __popc(eq_ballot & ((1u << lane) - 1u));
-            const bool sel = (j < Tb) && (k > thr || (eq && eq_rank < eq_left) || j >= mg.sink_first);
-            eq_left -= __popc(eq_ballot);
-            const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
-            if (sel) out[written + __popc(sel_ballot & ((1u << lane) - 1u))] = j;
-            written += __popc(sel_ballot);
-        }
-        if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = written; }
-    }
+    for (int r = warp; r < nrows; r += kSelThreads / 32)
+        select_row(keys + (size_t)r * Tb, hist, mg, bh, i0 + r, lane, row_start, row_count, col_idx, keep_all);
 }
 
 }  // namespace rf2

@@ -52,6 +52,7 @@ static Checked check_geometry(const rf2_geometry* g)
     if (g->block != kBlock) return c;
     const int64_t Tb = (N + kBlock - 1) / kBlock;
     if (Tb > kMaxBlocks) return c;
+    if ((int64_t)2 * g->batch * g->heads * Tb > INT32_MAX) return c;   // block-mean rows index a TMA map
     c.BH = (int64_t)g->batch * g->heads;
     if (c.BH > (int64_t)INT32_MAX / 2) return c;
     c.N = (int32_t)N;
@@ -72,6 +73,17 @@ static int keep_count(double keep, int32_t Tb, int32_t* n)
     return RF2_OK;
 }
 
+// Mask-prediction workspace: the block means as a tf32 hi/lo split, two
+// fp32 arrays [2][BH][T_b][d], then the pooled-score buffer of one group of
+// heads [G][T_b][ld] (ld = T_b rounded up to 4 floats); heads are scored and
+// selected group by group so that the score buffer stays in L2 between the
+// two kernels.
+constexpr int64_t kScoreGroupHeads = 16;
+static int32_t score_ld(int32_t Tb) { return (Tb + 3) & ~3; }
+static size_t mask_means_bytes(const Checked& c) { return ((size_t)2 * c.BH * c.Tb * c.D * sizeof(float) + 255) & ~(size_t)255; }
+static size_t score_head_bytes(const Checked& c) { return (size_t)c.Tb * score_ld(c.Tb) * sizeof(float); }
+static int64_t score_group_heads(int64_t BH) { return BH < kScoreGroupHeads ? BH : kScoreGroupHeads; }
+
 static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg, rf2_sizes* out)
 {
     c = check_geometry(g);
@@ -90,7 +102,7 @@ static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg
         out->row_capacity = mg.cap;
         out->num_rows = c.BH * c.Tb;
         out->col_idx_capacity = total;
-        out->mask_workspace_bytes = (size_t)2 * c.BH * c.Tb * c.D * sizeof(float);
+        out->mask_workspace_bytes = 2 * mask_means_bytes(c) + (size_t)score_group_heads(c.BH) * score_head_bytes(c);
     }
     return RF2_OK;
 }
@@ -227,18 +239,98 @@ static int launch_attn(const Checked& c, const MaskGeo& mg, const void* qp, cons
     return launch_status();
 }
 
-template <int D, int R>
-static int launch_select(const Checked& c, const MaskGeo& mg, const float* means, int32_t* row_start,
-                         int32_t* row_count, int32_t* col_idx, cudaStream_t s)
+// The [2*BH*T_b, d] fp32 block-mean array (hi or lo part) as a 2D tensor map:
+// box = 32 floats (128 bytes) x `box_rows` rows, 128-byte swizzle (K-major
+// tf32 tiles).
+static bool make_means_map(CUtensorMap* m, const float* ptr, int32_t D, int64_t rows, uint32_t box_rows)
 {
-    const size_t smem = SelectSmem<D, R>::bytes(c.Tb);
-    if (cudaFuncSetAttribute(select_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+    const cuuint32_t box[2] = {32, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int num_sms()
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+template <int D>
+static int launch_scores(const Checked& c, const float* means_hi, const float* means_lo, float* S, int64_t h0,
+                         int64_t g, cudaStream_t s)
+{
+    using Cfg = ScoreCfg<D>;
+    int* status = status_word_ptr();
+    if (!status) return RF2_ERR_CUDA;
+    const int64_t rows = 2 * c.BH * c.Tb;
+    CUtensorMap mh, ml, mhb, mlb;
+    if (!make_means_map(&mh, means_hi, D, rows, 128) || !make_means_map(&ml, means_lo, D, rows, 128) ||
+        !make_means_map(&mhb, means_hi, D, rows, Cfg::NCH) || !make_means_map(&mlb, means_lo, D, rows, Cfg::NCH))
+        return RF2_ERR_CUDA;
+    if (cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) !=
         cudaSuccess)
         return RF2_ERR_CUDA;
-    dim3 grid((c.Tb + R - 1) / R, (unsigned)c.BH);
-    select_kernel<D, R><<<grid, kSelThreads, smem, s>>>(means, row_start, row_count, col_idx, mg, c.BH,
-                                                       (float)(1.0 / sqrt((double)D)));
+    const int64_t items = g * ((c.Tb + 127) / 128);
+    const int grid = (int)(items < num_sms() ? items : num_sms());
+    score_tc_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM, s>>>(mh, ml, mhb, mlb, S, c.Tb, score_ld(c.Tb), c.BH, h0,
+                                                             (int32_t)g, (float)(1.0 / sqrt((double)D)), status);
     return launch_status();
+}
+
+template <int R>
+static int launch_select(const Checked& c, const MaskGeo& mg, const float* S, int64_t h0, int64_t g,
+                         int32_t* row_start, int32_t* row_count, int32_t* col_idx, cudaStream_t s)
+{
+    const size_t smem = sizeof(uint32_t) * ((size_t)R * c.Tb + 256 * (kSelThreads / 32));
+    if (cudaFuncSetAttribute(select_from_scores_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return RF2_ERR_CUDA;
+    dim3 grid((c.Tb + R - 1) / R, (unsigned)g);
+    select_from_scores_kernel<R><<<grid, kSelThreads, smem, s>>>(S, score_ld(c.Tb), row_start, row_count,
+                                                                 col_idx, mg, h0);
+    return launch_status();
+}
+
+// Block means, then per group of heads the tensor-core scores and the
+// selection.  `ws` holds the means followed by a score buffer for as many
+// heads (at most kScoreGroupHeads) as `ws_bytes` allows.
+static int launch_mask(const Checked& c, const MaskGeo& mg, const void* qp, const void* kp, int32_t* row_start,
+                       int32_t* row_count, int32_t* col_idx, void* ws, size_t ws_bytes, cudaStream_t s)
+{
+    const size_t mb = mask_means_bytes(c);
+    if (ws_bytes < 2 * mb + score_head_bytes(c)) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    int64_t G = (int64_t)((ws_bytes - 2 * mb) / score_head_bytes(c));
+    if (G > score_group_heads(c.BH)) G = score_group_heads(c.BH);
+    float* means_hi = reinterpret_cast<float*>(ws);
+    float* means_lo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + mb);
+    float* S = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 2 * mb);
+    const int64_t warps = 2 * c.BH * c.Tb;
+    const unsigned grid = (unsigned)((warps + 7) / 8);
+    if (c.D == 128)
+        block_mean_kernel<128><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
+                                                     reinterpret_cast<const uint4*>(kp), means_hi, means_lo, c.N,
+                                                     c.Tb, c.BH);
+    else
+        block_mean_kernel<64><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
+                                                    reinterpret_cast<const uint4*>(kp), means_hi, means_lo, c.N,
+                                                    c.Tb, c.BH);
+    int r = launch_status();
+    for (int64_t h0 = 0; r == RF2_OK && h0 < c.BH; h0 += G) {
+        const int64_t g = (c.BH - h0 < G) ? c.BH - h0 : G;
+        r = (c.D == 128) ? launch_scores<128>(c, means_hi, means_lo, S, h0, g, s)
+                         : launch_scores<64>(c, means_hi, means_lo, S, h0, g, s);
+        if (r != RF2_OK) break;
+        r = launch_select<8>(c, mg, S, h0, g, row_start, row_count, col_idx, s);
+    }
+    return r;
 }
 
 // ------------------------------------------------------------------------
@@ -328,25 +420,8 @@ int rf2_predict_mask(const rf2_geometry* geom, const void* qp, const void* kp, d
         !aligned16(row_count) || !aligned16(col_idx))
         return RF2_ERR_INVALID_ARGUMENT;
     if (workspace_bytes < sz.mask_workspace_bytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    float* means = reinterpret_cast<float*>(workspace);
-    const int64_t warps = 2 * c.BH * c.Tb;
-    const unsigned grid = (unsigned)((warps + 7) / 8);
-    if (c.D == 128)
-        block_mean_kernel<128><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
-                                                     reinterpret_cast<const uint4*>(kp), means, c.N, c.Tb, c.BH);
-    else
-        block_mean_kernel<64><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
-                                                    reinterpret_cast<const uint4*>(kp), means, c.N, c.Tb, c.BH);
-    int r = launch_status();
-    if (r != RF2_OK) return r;
-    if (c.Tb <= 2048)
-        r = (c.D == 128) ? launch_select<128, 16>(c, mg, means, row_start, row_count, col_idx, s)
-                         : launch_select<64, 16>(c, mg, means, row_start, row_count, col_idx, s);
-    else
-        r = (c.D == 128) ? launch_select<128, 8>(c, mg, means, row_start, row_count, col_idx, s)
-                         : launch_select<64, 8>(c, mg, means, row_start, row_count, col_idx, s);
-    return r;
+    return launch_mask(c, mg, qp, kp, row_start, row_count, col_idx, workspace, workspace_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 int rf2_block_sparse_attn(const rf2_geometry* geom, const void* qp, const void* kp, const void* vp,
@@ -376,30 +451,15 @@ int rf2_predict_mask_static(const rf2_geometry* geom, const void* qp, const void
     if (!qp || !kp || !row_start || !row_count || !col_idx) return RF2_ERR_INVALID_ARGUMENT;
     if (!aligned16(qp) || !aligned16(kp) || !aligned16(row_start) || !aligned16(row_count) || !aligned16(col_idx))
         return RF2_ERR_INVALID_ARGUMENT;
-    if (sz.mask_workspace_bytes > kStaticScratchBytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
-    float* means = nullptr;
-    const int ss = static_scratch(&means);
+    // Needs room for the block means and the scores of at least one head.
+    if (2 * mask_means_bytes(c) + score_head_bytes(c) > kStaticScratchBytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    float* scratch = nullptr;
+    const int ss = static_scratch(&scratch);
     if (ss != RF2_OK) return ss;
-    // The block means fill every scratch element the select kernel reads, so
-    // nothing left from an earlier call needs clearing.
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t warps = 2 * c.BH * c.Tb;
-    const unsigned grid = (unsigned)((warps + 7) / 8);
-    if (c.D == 128)
-        block_mean_kernel<128><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
-                                                     reinterpret_cast<const uint4*>(kp), means, c.N, c.Tb, c.BH);
-    else
-        block_mean_kernel<64><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
-                                                    reinterpret_cast<const uint4*>(kp), means, c.N, c.Tb, c.BH);
-    int r = launch_status();
-    if (r != RF2_OK) return r;
-    if (c.Tb <= 2048)
-        r = (c.D == 128) ? launch_select<128, 16>(c, mg, means, row_start, row_count, col_idx, s)
-                         : launch_select<64, 16>(c, mg, means, row_start, row_count, col_idx, s);
-    else
-        r = (c.D == 128) ? launch_select<128, 8>(c, mg, means, row_start, row_count, col_idx, s)
-                         : launch_select<64, 8>(c, mg, means, row_start, row_count, col_idx, s);
-    return r;
+    // Every scratch element the kernels read is written earlier in the same
+    // call, so nothing left from an earlier call needs clearing.
+    return launch_mask(c, mg, qp, kp, row_start, row_count, col_idx, scratch, kStaticScratchBytes,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 int rf2_device_status(void* stream)

@@ -74,7 +74,9 @@ typedef struct {
     int32_t row_capacity;        /* col_idx slots of a non-sink row: min(T_b, n_keep + sink blocks) */
     int64_t num_rows;            /* batch * heads * T_b: length of row_start / row_count */
     int64_t col_idx_capacity;    /* length of col_idx */
-    size_t  mask_workspace_bytes;/* scratch for rf2_predict_mask (block means, fp32) */
+    size_t  mask_workspace_bytes;/* scratch for rf2_predict_mask: the block means as a
+                                    tf32 hi/lo pair of fp32 arrays, then the pooled
+                                    scores of up to 16 heads at a time */
 } rf2_sizes;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -100,7 +102,8 @@ int rf2_unpermute(const rf2_geometry* geom, const void* xp_bf16, void* x_bf16, v
 
 /* Online block-mask prediction (section 3.2, eqs. (5)-(8), and section 3.4).
  *   q^_i = mean of the valid rows of query block i (fp32), likewise k^_j;
- *   S^_ij = q^_i . k^_j / sqrt(d) (fp32);
+ *   S^_ij = q^_i . k^_j / sqrt(d) (tensor cores, tf32 hi/lo split: about
+ *           2^-21 relative error, i.e. fp32 accuracy);
  *   a non-sink row keeps its n_keep largest S^_ij (equal scores: lower j
  *   first) plus every sink column; a sink row keeps every column.
  * Output is one CSR row per (b, h, i), r = (b*heads + h)*T_b + i:
@@ -122,11 +125,12 @@ int rf2_predict_mask(const rf2_geometry* geom, const void* qp_bf16, const void* 
  * owns the device allocator and hands out no workspace, or a latency-critical
  * loop where cudaMalloc's implicit device synchronization is not acceptable.
  * (The paper has no counterpart to this call; it exists only for such callers.)
- * - Limit: 2*batch*heads*T_b*head_dim*4 bytes (rf2_sizes.mask_workspace_bytes)
- *   must not exceed 64 MiB (67,108,864), i.e. batch*heads <= 55 at 720p
- *   (75,600 tokens, d = 128); larger problems return
- *   RF2_ERR_INSUFFICIENT_WORKSPACE and launch nothing (split the heads over
- *   several calls, or use rf2_predict_mask).
+ * - Limit: the block means as a hi/lo pair (2 x 2*batch*heads*T_b*head_dim*4
+ *   bytes) plus the pooled scores of one head (T_b*ceil4(T_b)*4 bytes) must
+ *   fit in 64 MiB (67,108,864), i.e. batch*heads <= 25 at 720p (75,600
+ *   tokens, d = 128);
+ *   larger problems return RF2_ERR_INSUFFICIENT_WORKSPACE and launch nothing
+ *   (split the heads over several calls, or use rf2_predict_mask).
  * - Every GPU that loads the library holds the 64 MiB until the process exits.
  * - The first call on a device looks up the array's device address (with that
  *   device current) and caches it; make that first call before any stream

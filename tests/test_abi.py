@@ -58,7 +58,9 @@ def test_query_matches_oracle_readings(L, name):
     assert sz.num_rows == BH * Tb
     s0 = Tb if sz.sink_first < 0 else sz.sink_first
     assert sz.col_idx_capacity == BH * (s0 * sz.row_capacity + (Tb - s0) * Tb)
-    assert sz.mask_workspace_bytes == 2 * BH * Tb * wl.head_dim * 4
+    means = (2 * BH * Tb * wl.head_dim * 4 + 255) // 256 * 256
+    scores_per_head = Tb * ((Tb + 3) // 4 * 4) * 4
+    assert sz.mask_workspace_bytes == 2 * means + min(BH, 16) * scores_per_head
 
 
 def test_keep_ratio_matches_oracle(L):

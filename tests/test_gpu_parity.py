@@ -88,6 +88,27 @@ def test_image_parity():
     assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, e
 
 
+@pytest.mark.parametrize("d,T,H,W", [(128, 3, 16, 24), (64, 2, 20, 21), (128, 1, 64, 64)])
+def test_pooled_scores_precision(d, T, H, W):
+    """The tensor-core pooled scores (tf32 hi/lo products) left in the mask
+    workspace agree with the fp64 oracle's S^ to well inside the 1e-5 band."""
+    rope = (0, d // 2, d // 2) if T == 1 else ((24, 20, 20) if d == 64 else (44, 42, 42))
+    wl = Workload("scores", 1, 3, d, T, H, W, 1, 8, 8, 0.3, T > 1, rope)
+    q, k, _ = make_qkv(wl, "cuda", seed=17)
+    g = rf2.geometry_of(wl)
+    qp, kp = rf2.permute(g, q), rf2.permute(g, k)
+    mask, ws = rf2.alloc_mask(g, wl.keep, qp.device)
+    rf2.predict_mask(g, qp, kp, wl.keep, mask, ws)
+    torch.cuda.synchronize()
+    Tb = wl.num_blocks
+    means_bytes = (2 * wl.heads * Tb * d * 4 + 255) // 256 * 256
+    ld = (Tb + 3) // 4 * 4
+    S_gpu = ws[2 * means_bytes:2 * means_bytes + wl.heads * Tb * ld * 4].view(torch.float32).view(wl.heads, Tb, ld)[..., :Tb]
+    S_ref = oracle.pooled_scores(oracle.block_means(bits(qp)), oracle.block_means(bits(kp)))[0]
+    err = np.abs(S_gpu.double().cpu().numpy() - S_ref)
+    assert err.max() <= 2e-6 * max(1.0, np.abs(S_ref).max()), (err.max(), np.abs(S_ref).max())
+
+
 def test_keep_all_equals_dense_attention():
     """keep = 1 selects every block: the output is dense softmax attention, and
     unpermuting it gives dense attention in the model's order."""
