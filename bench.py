@@ -167,10 +167,12 @@ def cpu_info():
     return model
 
 
-def oracle_sample(wl, seed=0, n_query_blocks=32):
+def oracle_sample(wl, seed=0, n_query_blocks=32, budget_s=None):
     """The oracle as it stands on one head of the workload: permutation of Q,
     K, V, the full mask of that head, and attention for a sample of query
-    blocks (one of them a sink block).  Returns (kept_flops, seconds, desc)."""
+    blocks (one of them a sink block).  With budget_s, attention runs in
+    chunks of n_query_blocks random query blocks until that many seconds have
+    passed.  Returns (kept_flops, seconds, desc)."""
     import oracle
     from image_dits_b200.workload import Workload
     one = Workload(wl.name, 1, 1, wl.head_dim, wl.frames, wl.height, wl.width, wl.win_t, wl.win_h, wl.win_w,
@@ -188,12 +190,20 @@ def oracle_sample(wl, seed=0, n_query_blocks=32):
     rng = np.random.default_rng(seed)
     s0 = oracle.sink_start(wl.frames, wl.height, wl.width, wl.sink)
     upper = s0 if s0 > 0 else Tb
-    blocks = list(rng.choice(upper, size=min(n_query_blocks - 1, upper), replace=False))
-    blocks.append(Tb - 1)
-    items = np.array([(0, int(i)) for i in blocks], dtype=np.int64)
+    order = [int(i) for i in rng.permutation(upper) if i != Tb - 1]
     N = wl.num_tokens
-    out, _ = oracle.masked_attention(qp.reshape(1, N, -1), kp.reshape(1, N, -1), vp.reshape(1, N, -1),
-                                     mask.reshape(1, Tb, Tb), items)
+    blocks = []
+    chunk = [Tb - 1] + order[:n_query_blocks - 1]
+    pos = n_query_blocks - 1
+    while chunk:
+        items = np.array([(0, i) for i in chunk], dtype=np.int64)
+        oracle.masked_attention(qp.reshape(1, N, -1), kp.reshape(1, N, -1), vp.reshape(1, N, -1),
+                                mask.reshape(1, Tb, Tb), items)
+        blocks += chunk
+        if budget_s is None or time.perf_counter() - t0 >= budget_s or pos >= len(order):
+            break
+        chunk = order[pos:pos + n_query_blocks]
+        pos += n_query_blocks
     oracle.unpermute(qp, perm)
     dt = time.perf_counter() - t0
     last = N - 64 * (Tb - 1)
@@ -282,25 +292,29 @@ def main():
     mask, ws = rf2.alloc_mask(g, wl.keep, dev)
     stream = torch.cuda.current_stream()
 
+    score_groups = -(-wl.batch * wl.heads // 16)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        rf2.permute(g, q, qp)
-        rf2.permute(g, k, kp)
-        rf2.permute(g, v, vp)
+        rf2.permute_qk_pool(g, q, k, ws, qp, kp)
         if ev is not None:
             ev[1].record(stream)
-        rf2.predict_mask(g, qp, kp, wl.keep, mask, ws)
+        rf2.permute(g, v, vp)
         if ev is not None:
             ev[2].record(stream)
-        rf2.block_sparse_attn(g, qp, kp, vp, mask, op)
+        rf2.predict_mask_pooled(g, wl.keep, mask, ws)
         if ev is not None:
             ev[3].record(stream)
-        rf2.unpermute(g, op, o)
+        rf2.block_sparse_attn(g, qp, kp, vp, mask, op)
         if ev is not None:
             ev[4].record(stream)
+        rf2.unpermute(g, op, o)
+        if ev is not None:
+            ev[5].record(stream)
 
-    launches_per_step = 7  # 3 permute + block means + select + attention + unpermute
+    # permute+pool, permute V, (scores + select) per group of 16 heads, attention, unpermute
+    launches_per_step = 2 + 2 * score_groups + 2
 
     for _ in range(args.warmup):
         step()
@@ -313,7 +327,7 @@ def main():
     density = kept_pairs / (wl.batch * wl.heads * Tb * Tb)
 
     sampler = ClockSampler(local_rank)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
@@ -328,8 +342,8 @@ def main():
     clocks = sampler.stop()
     total_ms = t_start.elapsed_time(t_end)
     stage_ms = {name: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
-                for name, a, b in (("permute_qkv", 0, 1), ("predict_mask", 1, 2), ("block_sparse_attn", 2, 3),
-                                   ("unpermute", 3, 4))}
+                for name, a, b in (("permute_qk_pool", 0, 1), ("permute_v", 1, 2), ("predict_mask_pooled", 2, 3),
+                                   ("block_sparse_attn", 3, 4), ("unpermute", 4, 5))}
     if rf2.device_status() != rf2.RF2_OK:
         raise RuntimeError("device status not ok after timing")
 
@@ -366,8 +380,11 @@ def main():
     peaks, peak_src = load_peaks()
     attn_tf = flops / (stage_ms["block_sparse_attn"] * 1e-3) / 1e12
     attn_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    mbytes = mask_bytes(wl, mask)
-    pbytes = 3 * 2 * q.numel() * 2
+    means = 2 * wl.batch * wl.heads * Tb * wl.head_dim * 4
+    qkbytes = 2 * 2 * q.numel() * 2 + 2 * means        # read Q, K; write Qp, Kp and the hi/lo means
+    vbytes = 2 * v.numel() * 2
+    csr = 4 * (2 * mask.row_count.numel() + mask.kept_pairs())
+    pbytes_mask = 2 * means + csr                       # read the means, write the CSR mask
     ubytes = 2 * o.numel() * 2
     hbm = peaks["hbm_gbs"]
 
@@ -375,10 +392,15 @@ def main():
         return b / (ms * 1e-3) / 1e9
 
     stages = {
-        "permute_qkv": {"ms": stage_ms["permute_qkv"], "GB/s": gbs(pbytes, stage_ms["permute_qkv"]),
-                        "bytes": pbytes, "frac": gbs(pbytes, stage_ms["permute_qkv"]) / hbm, "bound": "hbm"},
-        "predict_mask": {"ms": stage_ms["predict_mask"], "GB/s": gbs(mbytes, stage_ms["predict_mask"]),
-                         "bytes": mbytes, "frac": gbs(mbytes, stage_ms["predict_mask"]) / hbm, "bound": "hbm"},
+        "permute_qk_pool": {"ms": stage_ms["permute_qk_pool"], "GB/s": gbs(qkbytes, stage_ms["permute_qk_pool"]),
+                            "bytes": qkbytes, "frac": gbs(qkbytes, stage_ms["permute_qk_pool"]) / hbm,
+                            "bound": "hbm"},
+        "permute_v": {"ms": stage_ms["permute_v"], "GB/s": gbs(vbytes, stage_ms["permute_v"]), "bytes": vbytes,
+                      "frac": gbs(vbytes, stage_ms["permute_v"]) / hbm, "bound": "hbm"},
+        "predict_mask_pooled": {"ms": stage_ms["predict_mask_pooled"], "bytes": pbytes_mask,
+                                "GB/s": gbs(pbytes_mask, stage_ms["predict_mask_pooled"]),
+                                "note": "scores + top-n selection from the pooled means; the Q/K read of mask "
+                                        "prediction is fused into permute_qk_pool"},
         "block_sparse_attn": {"ms": stage_ms["block_sparse_attn"], "TFLOP/s": attn_tf, "flops": flops,
                               "frac": attn_tf / attn_peak, "bound": "tensor"},
         "unpermute": {"ms": stage_ms["unpermute"], "GB/s": gbs(ubytes, stage_ms["unpermute"]), "bytes": ubytes,
@@ -417,6 +439,22 @@ def main():
                        "ms_per_step": e2e_ms_all, "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                        "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]}
 
+    # mask prediction as one call on the permuted Q/K (Q and K read again), for its HBM roofline
+    for _ in range(3):
+        rf2.predict_mask(g, qp, kp, wl.keep, mask, ws)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(5):
+        rf2.predict_mask(g, qp, kp, wl.keep, mask, ws)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_pm = a.elapsed_time(b) / 5
+    mbytes = mask_bytes(wl, mask)
+    stages["predict_mask_unfused"] = {"ms": ms_pm, "GB/s": gbs(mbytes, ms_pm), "bytes": mbytes,
+                                      "frac": gbs(mbytes, ms_pm) / hbm, "bound": "hbm",
+                                      "note": "rf2_predict_mask outside the step: reads Qp, Kp"}
+
     if args.sweep and rank == 0:
         sweep = []
         for keep in SWEEP_KEEPS:
@@ -452,7 +490,7 @@ def main():
         try:
             import oracle
             oracle.build()
-            f, dt, desc = oracle_sample(wl)
+            f, dt, desc = oracle_sample(wl, budget_s=12.0)
             line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                                     "kind": "oracle", "cpu": cpu_info(), "seconds": dt, "sample": desc}
         except Exception as exc:  # the baseline must not hide the GPU line

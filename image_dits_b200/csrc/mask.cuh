@@ -84,6 +84,88 @@ __global__ void __launch_bounds__(256) block_mean_kernel(const uint4* __restrict
     }
 }
 
+// Permutation of Q and K fused with the block means (the "permute + pooling"
+// step): warp w takes 64-row blocks of the permuted output of both tensors
+// (blocks 0 .. BH*Tb-1 of Q, then those of K), copies each block's rows in
+// batches of 16 rows (8 at d = 128) as permute_rows_kernel does, and
+// accumulates the block's column sums in registers in the same row order as
+// block_mean_kernel, so the means (and the masks predicted from them) are
+// bit-identical to the unfused path.  Saves re-reading Qp and Kp.
+#ifndef RF2_POOL_SUB
+#define RF2_POOL_SUB 8
+#endif
+#ifndef RF2_POOL_MINB
+#define RF2_POOL_MINB 4
+#endif
+
+template <int D>
+__global__ void __launch_bounds__(256, D == 128 ? RF2_POOL_MINB : 4) permute_pool_kernel(
+    const uint4* __restrict__ q, const uint4* __restrict__ k, uint4* __restrict__ qp, uint4* __restrict__ kp,
+    PermGeo g, int32_t Tb, int64_t BH, float* __restrict__ means_hi, float* __restrict__ means_lo)
+{
+    constexpr int C = D / 8;          // 16-byte chunks per row
+    constexpr int R = 32 / C;         // rows covered by one warp-wide load
+    constexpr int kSub = D == 128 ? RF2_POOL_SUB : 16;   // rows per batch
+    constexpr int kLoads = kSub / R;
+    static_assert(kBlock % kSub == 0 && kSub % R == 0 && kSub <= 32, "rows per batch");
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int cidx = lane % C;
+    const int rsub = lane / C;
+    const int64_t per_tensor = BH * Tb;
+    const int32_t N = g.N;
+    for (int64_t blk = warp; blk < 2 * per_tensor; blk += nwarps) {
+        const int which = (int)(blk / per_tensor);
+        const int64_t rem = blk - which * per_tensor;
+        const int64_t bh = rem / Tb;
+        const int32_t i = (int32_t)(rem - bh * Tb);
+        const uint4* in = (which ? k : q) + bh * N * C + cidx;
+        uint4* out = (which ? kp : qp) + (bh * N + (int64_t)i * kBlock) * C + cidx;
+        const int32_t rows = min(kBlock, N - i * kBlock);
+        float acc[8];
+        #pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+        #pragma unroll 1
+        for (int r0 = 0; r0 < rows; r0 += kSub) {
+            int32_t src = 0;
+            if (lane < kSub && r0 + lane < rows) src = perm_src(g, i * kBlock + r0 + lane);
+            uint4 v[kLoads];
+            #pragma unroll
+            for (int u = 0; u < kLoads; ++u) {
+                const int r = u * R + rsub;
+                const int32_t srow = __shfl_sync(0xffffffffu, src, r);
+                if (r0 + r < rows) v[u] = __ldcs(in + (int64_t)srow * C);
+            }
+            #pragma unroll
+            for (int u = 0; u < kLoads; ++u) {
+                const int r = r0 + u * R + rsub;
+                if (r < rows) {
+                    __stcs(out + r * C, v[u]);
+                    bf16x8_accumulate(v[u], acc);
+                }
+            }
+        }
+        #pragma unroll
+        for (int off = C; off < 32; off <<= 1)
+            #pragma unroll
+            for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], off);
+        if (lane < C) {
+            const float fr = (float)rows;
+            const int64_t at = ((int64_t)which * per_tensor + rem) * D + 8 * cidx;
+            float m[8], h[8];
+            #pragma unroll
+            for (int c = 0; c < 8; ++c) { m[c] = acc[c] / fr; h[c] = to_tf32(m[c]); }
+            float4* dh = reinterpret_cast<float4*>(means_hi + at);
+            float4* dl = reinterpret_cast<float4*>(means_lo + at);
+            dh[0] = make_float4(h[0], h[1], h[2], h[3]);
+            dh[1] = make_float4(h[4], h[5], h[6], h[7]);
+            dl[0] = make_float4(m[0] - h[0], m[1] - h[1], m[2] - h[2], m[3] - h[3]);
+            dl[1] = make_float4(m[4] - h[4], m[5] - h[5], m[6] - h[6], m[7] - h[7]);
+        }
+    }
+}
+
 // Order-preserving map float -> uint32 (larger float, larger key).
 __device__ __forceinline__ uint32_t float_order_key(float f)
 {

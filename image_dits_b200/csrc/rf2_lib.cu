@@ -302,35 +302,62 @@ static int launch_select(const Checked& c, const MaskGeo& mg, const float* S, in
 // Block means, then per group of heads the tensor-core scores and the
 // selection.  `ws` holds the means followed by a score buffer for as many
 // heads (at most kScoreGroupHeads) as `ws_bytes` allows.
-static int launch_mask(const Checked& c, const MaskGeo& mg, const void* qp, const void* kp, int32_t* row_start,
-                       int32_t* row_count, int32_t* col_idx, void* ws, size_t ws_bytes, cudaStream_t s)
+// Workspace pointers of the mask path; G = heads scored per group.
+struct MaskWs {
+    float* means_hi;
+    float* means_lo;
+    float* S;
+    int64_t G;
+};
+
+static int mask_ws(const Checked& c, void* ws, size_t ws_bytes, MaskWs* w)
 {
     const size_t mb = mask_means_bytes(c);
     if (ws_bytes < 2 * mb + score_head_bytes(c)) return RF2_ERR_INSUFFICIENT_WORKSPACE;
     int64_t G = (int64_t)((ws_bytes - 2 * mb) / score_head_bytes(c));
     if (G > score_group_heads(c.BH)) G = score_group_heads(c.BH);
-    float* means_hi = reinterpret_cast<float*>(ws);
-    float* means_lo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + mb);
-    float* S = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 2 * mb);
+    w->means_hi = reinterpret_cast<float*>(ws);
+    w->means_lo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + mb);
+    w->S = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 2 * mb);
+    w->G = G;
+    return RF2_OK;
+}
+
+// Per group of heads: the tensor-core scores, then the selection.
+static int launch_score_select(const Checked& c, const MaskGeo& mg, const MaskWs& w, int32_t* row_start,
+                               int32_t* row_count, int32_t* col_idx, cudaStream_t s)
+{
+    int r = RF2_OK;
+    for (int64_t h0 = 0; r == RF2_OK && h0 < c.BH; h0 += w.G) {
+        const int64_t g = (c.BH - h0 < w.G) ? c.BH - h0 : w.G;
+        r = (c.D == 128) ? launch_scores<128>(c, w.means_hi, w.means_lo, w.S, h0, g, s)
+                         : launch_scores<64>(c, w.means_hi, w.means_lo, w.S, h0, g, s);
+        if (r != RF2_OK) break;
+        r = launch_select<8>(c, mg, w.S, h0, g, row_start, row_count, col_idx, s);
+    }
+    return r;
+}
+
+// Block means of the permuted Q and K, then scores and selection.
+static int launch_mask(const Checked& c, const MaskGeo& mg, const void* qp, const void* kp, int32_t* row_start,
+                       int32_t* row_count, int32_t* col_idx, void* ws, size_t ws_bytes, cudaStream_t s)
+{
+    MaskWs w;
+    const int st = mask_ws(c, ws, ws_bytes, &w);
+    if (st != RF2_OK) return st;
     const int64_t warps = 2 * c.BH * c.Tb;
     const unsigned grid = (unsigned)((warps + 7) / 8);
     if (c.D == 128)
         block_mean_kernel<128><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
-                                                     reinterpret_cast<const uint4*>(kp), means_hi, means_lo, c.N,
-                                                     c.Tb, c.BH);
+                                                     reinterpret_cast<const uint4*>(kp), w.means_hi, w.means_lo,
+                                                     c.N, c.Tb, c.BH);
     else
         block_mean_kernel<64><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
-                                                    reinterpret_cast<const uint4*>(kp), means_hi, means_lo, c.N,
-                                                    c.Tb, c.BH);
-    int r = launch_status();
-    for (int64_t h0 = 0; r == RF2_OK && h0 < c.BH; h0 += G) {
-        const int64_t g = (c.BH - h0 < G) ? c.BH - h0 : G;
-        r = (c.D == 128) ? launch_scores<128>(c, means_hi, means_lo, S, h0, g, s)
-                         : launch_scores<64>(c, means_hi, means_lo, S, h0, g, s);
-        if (r != RF2_OK) break;
-        r = launch_select<8>(c, mg, S, h0, g, row_start, row_count, col_idx, s);
-    }
-    return r;
+                                                    reinterpret_cast<const uint4*>(kp), w.means_hi, w.means_lo,
+                                                    c.N, c.Tb, c.BH);
+    const int r = launch_status();
+    if (r != RF2_OK) return r;
+    return launch_score_select(c, mg, w, row_start, row_count, col_idx, s);
 }
 
 // ------------------------------------------------------------------------
@@ -460,6 +487,56 @@ int rf2_predict_mask_static(const rf2_geometry* geom, const void* qp, const void
     // call, so nothing left from an earlier call needs clearing.
     return launch_mask(c, mg, qp, kp, row_start, row_count, col_idx, scratch, kStaticScratchBytes,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int rf2_permute_qk_pool(const rf2_geometry* geom, const void* q, const void* k, void* qp, void* kp,
+                        void* workspace, size_t workspace_bytes, void* stream)
+{
+    Checked c;
+    MaskGeo mg;
+    rf2_sizes sz;
+    const int st = sizes_for(geom, 1.0, c, mg, &sz);
+    if (st != RF2_OK) return st;
+    if (!q || !k || !qp || !kp || !workspace) return RF2_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(qp) || !aligned16(kp) || !aligned16(workspace))
+        return RF2_ERR_INVALID_ARGUMENT;
+    if (q == qp || k == kp || q == kp || k == qp) return RF2_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < sz.mask_workspace_bytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    MaskWs w;
+    const int ws_st = mask_ws(c, workspace, workspace_bytes, &w);
+    if (ws_st != RF2_OK) return ws_st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t blocks = 2 * c.BH * c.Tb;
+    int64_t grid = (blocks + 7) / 8;
+    const int64_t cap = (int64_t)num_sms() * 16;
+    if (grid > cap) grid = cap;
+    if (c.D == 128)
+        permute_pool_kernel<128><<<(unsigned)grid, 256, 0, s>>>(
+            reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), reinterpret_cast<uint4*>(qp),
+            reinterpret_cast<uint4*>(kp), c.pg, c.Tb, c.BH, w.means_hi, w.means_lo);
+    else
+        permute_pool_kernel<64><<<(unsigned)grid, 256, 0, s>>>(
+            reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), reinterpret_cast<uint4*>(qp),
+            reinterpret_cast<uint4*>(kp), c.pg, c.Tb, c.BH, w.means_hi, w.means_lo);
+    return launch_status();
+}
+
+int rf2_predict_mask_pooled(const rf2_geometry* geom, double keep_ratio, int32_t* row_start, int32_t* row_count,
+                            int32_t* col_idx, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Checked c;
+    MaskGeo mg;
+    rf2_sizes sz;
+    const int st = sizes_for(geom, keep_ratio, c, mg, &sz);
+    if (st != RF2_OK) return st;
+    if (!row_start || !row_count || !col_idx || !workspace) return RF2_ERR_INVALID_ARGUMENT;
+    if (!aligned16(workspace) || !aligned16(row_start) || !aligned16(row_count) || !aligned16(col_idx))
+        return RF2_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < sz.mask_workspace_bytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    MaskWs w;
+    const int ws_st = mask_ws(c, workspace, workspace_bytes, &w);
+    if (ws_st != RF2_OK) return ws_st;
+    return launch_score_select(c, mg, w, row_start, row_count, col_idx, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int rf2_device_status(void* stream)

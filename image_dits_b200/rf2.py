@@ -26,7 +26,8 @@ RF2_ERR_TIMEOUT = 5
 # Every entry point declared in include/rf2.h.
 EXPORTED = (
     "rf2_status_string", "rf2_query", "rf2_permutation_index", "rf2_permute", "rf2_unpermute",
-    "rf2_predict_mask", "rf2_predict_mask_static", "rf2_block_sparse_attn", "rf2_device_status",
+    "rf2_predict_mask", "rf2_predict_mask_static", "rf2_permute_qk_pool", "rf2_predict_mask_pooled",
+    "rf2_block_sparse_attn", "rf2_device_status",
 )
 
 
@@ -75,6 +76,8 @@ def lib():
         L.rf2_unpermute.argtypes = [G, vp, vp, vp]
         L.rf2_predict_mask.argtypes = [G, vp, vp, f64, vp, vp, vp, vp, sz, vp]
         L.rf2_predict_mask_static.argtypes = [G, vp, vp, f64, vp, vp, vp, vp]
+        L.rf2_permute_qk_pool.argtypes = [G, vp, vp, vp, vp, vp, sz, vp]
+        L.rf2_predict_mask_pooled.argtypes = [G, f64, vp, vp, vp, vp, sz, vp]
         L.rf2_block_sparse_attn.argtypes = [G, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.rf2_device_status.argtypes = [vp]
         for name in EXPORTED:
@@ -193,6 +196,29 @@ def predict_mask(geom: Geometry, qp: torch.Tensor, kp: torch.Tensor, keep: float
     return mask
 
 
+def permute_qk_pool(geom: Geometry, q: torch.Tensor, k: torch.Tensor, workspace: torch.Tensor,
+                    qp: torch.Tensor | None = None, kp: torch.Tensor | None = None, stream=None):
+    """Permute Q and K and leave their block means in the mask workspace."""
+    _check_qkv(geom, q, k)
+    qp = torch.empty_like(q) if qp is None else qp
+    kp = torch.empty_like(k) if kp is None else kp
+    _check_qkv(geom, qp, kp)
+    _check(lib().rf2_permute_qk_pool(ctypes.byref(geom), q.data_ptr(), k.data_ptr(), qp.data_ptr(), kp.data_ptr(),
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)), "rf2_permute_qk_pool")
+    return qp, kp
+
+
+def predict_mask_pooled(geom: Geometry, keep: float, mask: BlockMask, workspace: torch.Tensor,
+                        stream=None) -> BlockMask:
+    """Mask prediction from the block means rf2_permute_qk_pool left in `workspace`."""
+    _check(lib().rf2_predict_mask_pooled(ctypes.byref(geom), float(keep), mask.row_start.data_ptr(),
+                                         mask.row_count.data_ptr(), mask.col_idx.data_ptr(), workspace.data_ptr(),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)),
+           "rf2_predict_mask_pooled")
+    return mask
+
+
 def block_sparse_attn(geom: Geometry, qp, kp, vp, mask: BlockMask, out: torch.Tensor | None = None,
                       lse: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     _check_qkv(geom, qp, kp, vp)
@@ -217,11 +243,12 @@ def device_status(stream=None) -> int:
 
 
 def rainfusion_attention(geom: Geometry, q, k, v, keep: float, stream=None):
-    """The whole path for one attention call: permute Q/K/V, predict the block
-    mask, block-sparse attention, unpermute.  Returns (O, mask)."""
-    qp = permute(geom, q, stream=stream)
-    kp = permute(geom, k, stream=stream)
+    """The whole path for one attention call: permute Q/K/V (block means of Q
+    and K taken on the way), predict the block mask, block-sparse attention,
+    unpermute.  Returns (O, mask)."""
+    mask, ws = alloc_mask(geom, keep, q.device)
+    qp, kp = permute_qk_pool(geom, q, k, ws, stream=stream)
     vp = permute(geom, v, stream=stream)
-    mask = predict_mask(geom, qp, kp, keep, stream=stream)
+    predict_mask_pooled(geom, keep, mask, ws, stream=stream)
     op = block_sparse_attn(geom, qp, kp, vp, mask, stream=stream)
     return unpermute(geom, op, stream=stream), mask

@@ -143,6 +143,23 @@ int rf2_predict_mask_static(const rf2_geometry* geom, const void* qp_bf16, const
                             double keep_ratio, int32_t* row_start, int32_t* row_count, int32_t* col_idx,
                             void* stream);
 
+/* The permutation of Q and K fused with the block means of mask prediction
+ * (sections 3.3-3.4 and eqs. (5)-(6)): writes Qp and Kp exactly as
+ * rf2_permute does, and the block means of Qp and Kp into `workspace`
+ * (a buffer of at least mask_workspace_bytes) while the rows pass through, so
+ * the mask step need not read Qp and Kp again.  Follow it with
+ * rf2_predict_mask_pooled on the same workspace; the masks equal those of
+ * rf2_permute + rf2_predict_mask bit for bit.  Inputs and outputs must not
+ * overlap. */
+int rf2_permute_qk_pool(const rf2_geometry* geom, const void* q_bf16, const void* k_bf16, void* qp_bf16,
+                        void* kp_bf16, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Mask prediction (section 3.2 eqs. (7)-(8), section 3.4) from the block
+ * means that rf2_permute_qk_pool left in `workspace`; outputs and errors as
+ * rf2_predict_mask. */
+int rf2_predict_mask_pooled(const rf2_geometry* geom, double keep_ratio, int32_t* row_start, int32_t* row_count,
+                            int32_t* col_idx, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Block-sparse FlashAttention forward (section 3.1): for every query block i,
  * O_i = softmax(Q_i K_J^T / sqrt(d)) V_J over the key blocks J kept in row i
  * of the CSR mask (eqs. (1)-(4); Q_i K_j^T and P_ij V_j are skipped when

@@ -24,12 +24,20 @@ def bf16_to_f64(b: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def run_path(geom, q, k, v, keep, lse=False):
-    """All four calls of one attention invocation; returns a dict of outputs."""
-    qp = rf2.permute(geom, q)
-    kp = rf2.permute(geom, k)
-    vp = rf2.permute(geom, v)
-    mask = rf2.predict_mask(geom, qp, kp, keep)
+def run_path(geom, q, k, v, keep, lse=False, fused=True):
+    """All calls of one attention invocation; returns a dict of outputs.
+    fused: Q/K permutation fused with the block means (rf2_permute_qk_pool +
+    rf2_predict_mask_pooled), else three rf2_permute calls + rf2_predict_mask."""
+    if fused:
+        mask, ws = rf2.alloc_mask(geom, keep, q.device)
+        qp, kp = rf2.permute_qk_pool(geom, q, k, ws)
+        vp = rf2.permute(geom, v)
+        rf2.predict_mask_pooled(geom, keep, mask, ws)
+    else:
+        qp = rf2.permute(geom, q)
+        kp = rf2.permute(geom, k)
+        vp = rf2.permute(geom, v)
+        mask = rf2.predict_mask(geom, qp, kp, keep)
     lse_t = None
     if lse:
         lse_t = torch.full((geom.batch * geom.heads * qp.shape[2],), float("nan"), device=q.device)

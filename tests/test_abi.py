@@ -124,6 +124,27 @@ def test_host_validation(L):
         rf2.RF2_ERR_INVALID_ARGUMENT
     assert L.rf2_predict_mask(G(good), fake, fake, 0.5, fake, fake, fake, ctypes.c_void_p(0x10004), 1 << 30,
                               None) == rf2.RF2_ERR_INVALID_ARGUMENT
+    # permute_qk_pool / predict_mask_pooled
+    f2, f3 = ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)
+    f4 = ctypes.c_void_p(0x40000)
+    big = 1 << 30
+    assert L.rf2_permute_qk_pool(G(good), fake, f2, f3, f4, ctypes.c_void_p(0x50000), ws_small, None) == \
+        rf2.RF2_ERR_INSUFFICIENT_WORKSPACE
+    assert L.rf2_permute_qk_pool(G(good), None, f2, f3, f4, fake, big, None) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_permute_qk_pool(G(good), fake, f2, fake, f4, ctypes.c_void_p(0x50000), big, None) == \
+        rf2.RF2_ERR_INVALID_ARGUMENT                                                  # in place
+    assert L.rf2_permute_qk_pool(G(good), fake, f2, f3, ctypes.c_void_p(0x40008), ctypes.c_void_p(0x50000), big,
+                                 None) == rf2.RF2_ERR_INVALID_ARGUMENT                # misaligned
+    assert L.rf2_permute_qk_pool(G(bad_dim), fake, f2, f3, f4, ctypes.c_void_p(0x50000), big, None) == \
+        rf2.RF2_ERR_UNSUPPORTED
+    assert L.rf2_predict_mask_pooled(G(good), 0.5, fake, fake, fake, fake, ws_small, None) == \
+        rf2.RF2_ERR_INSUFFICIENT_WORKSPACE
+    assert L.rf2_predict_mask_pooled(G(good), 0.0, fake, fake, fake, fake, big, None) == \
+        rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_predict_mask_pooled(G(good), 0.5, fake, None, fake, fake, big, None) == \
+        rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_predict_mask_pooled(G(good), 0.5, fake, fake, fake, None, big, None) == \
+        rf2.RF2_ERR_INVALID_ARGUMENT
     # block_sparse_attn
     assert L.rf2_block_sparse_attn(G(good), fake, fake, None, fake, fake, fake, fake, None, None) == \
         rf2.RF2_ERR_INVALID_ARGUMENT

@@ -132,6 +132,42 @@ def test_constant_value_rows():
     assert err <= 2 ** -7 * v.float().abs().max().item() + 1e-6
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged_d128", "ragged_d64_nosink", "one_block", "single_frame_sink",
+                                  "odd_blocks", "video720p"])
+def test_fused_permute_pool_matches_unfused(name):
+    """rf2_permute_qk_pool writes the same Qp/Kp as rf2_permute and the same
+    block means as the mask path's own pooling, bit for bit, so the predicted
+    masks are identical."""
+    wl = WORKLOADS[name] if name in WORKLOADS else dict(_small_cases())[name]
+    q, k, _ = make_qkv(wl, "cuda", seed=9)
+    g = rf2.geometry_of(wl)
+    mask_a, ws_a = rf2.alloc_mask(g, wl.keep, q.device)
+    qp_a, kp_a = rf2.permute_qk_pool(g, q, k, ws_a)
+    rf2.predict_mask_pooled(g, wl.keep, mask_a, ws_a)
+    qp_b, kp_b = rf2.permute(g, q), rf2.permute(g, k)
+    mask_b, ws_b = rf2.alloc_mask(g, wl.keep, q.device)
+    rf2.predict_mask(g, qp_b, kp_b, wl.keep, mask_b, ws_b)
+    torch.cuda.synchronize()
+    assert rf2.device_status() == rf2.RF2_OK
+    assert torch.equal(qp_a.view(torch.int16), qp_b.view(torch.int16))
+    assert torch.equal(kp_a.view(torch.int16), kp_b.view(torch.int16))
+    Tb = wl.num_blocks
+    means_bytes = (2 * wl.batch * wl.heads * Tb * wl.head_dim * 4 + 255) // 256 * 256
+    assert torch.equal(ws_a[:2 * means_bytes], ws_b[:2 * means_bytes])
+    assert torch.equal(mask_a.row_count, mask_b.row_count)
+    assert torch.equal(mask_a.row_start, mask_b.row_start)
+    assert np.array_equal(mask_a.dense(), mask_b.dense())
+    if name != "video720p":
+        perm = _perm_of(wl)
+        assert np.array_equal(bits(kp_a), oracle.permute(bits(k), perm))
+        hi = ws_a[:means_bytes].view(torch.float32)[:2 * wl.batch * wl.heads * Tb * wl.head_dim]
+        lo = ws_a[means_bytes:2 * means_bytes].view(torch.float32)[:hi.numel()]
+        m = (hi.double() + lo.double()).view(2, wl.batch * wl.heads, Tb, wl.head_dim).cpu().numpy()
+        m_ref = oracle.block_means(bits(kp_a).reshape(wl.batch * wl.heads, -1, wl.head_dim))
+        # fp32 sums of bf16 rows over at most 64 rows: relative 64 * 2^-24.
+        assert np.abs(m[1] - m_ref).max() <= 4e-6 * max(1.0, np.abs(m_ref).max())
+
+
 def test_deterministic():
     wl = WORKLOADS["tiny"]
     q, k, v = make_qkv(wl, "cuda", seed=11)
