@@ -373,6 +373,8 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tmem_ld32(s_row + 64 * g, a);
                 tmem_ld32(s_row + 64 * g + 32, b);
                 tmem_wait_ld();
+                reg_fence(a);
+                reg_fence(b);
                 if (nv[g] == 64) {
                     mx = max_chunk<false>(a, 64, mx);
                     mx = max_chunk<false>(b, 64, mx);
@@ -392,6 +394,7 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_addr + Cfg::TM_O + c0, o);
                     tmem_wait_ld();
+                    reg_fence(o);
                     #pragma unroll
                     for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
                     tmem_st32(tmem + lane_addr + Cfg::TM_O + c0, o);
@@ -409,12 +412,14 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                     uint32_t a[32];
                     tmem_ld32(s_row + 64 * g, a);
                     tmem_wait_ld();
+                    reg_fence(a);
                     uint32_t b[32];
                     tmem_ld32(s_row + 64 * g + 32, b);         // in flight during the first half
                     if (nv[g] == 64) exp_chunk<false>(a, sl2, neg_mu, 32, pk, sum4);
                     else exp_chunk<true>(a, sl2, neg_mu, nv[g], pk, sum4);
                     tmem_st16(s_row + 32 * g, pk);
                     tmem_wait_ld();
+                    reg_fence(b);
                     if (nv[g] == 64) exp_chunk<false>(b, sl2, neg_mu, 32, pk, sum4);
                     else exp_chunk<true>(b, sl2, neg_mu, nv[g] - 32, pk, sum4);
                     tmem_st16(s_row + 32 * g + 16, pk);
@@ -446,6 +451,7 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (T > 0) {
                     tmem_ld32(tmem + lane_addr + Cfg::TM_O + c0, o);
                     tmem_wait_ld();
+                    reg_fence(o);
                 } else {
                     #pragma unroll
                     for (int c = 0; c < 32; ++c) o[c] = 0u;

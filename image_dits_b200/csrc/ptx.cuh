@@ -233,6 +233,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// After tcgen05.wait::ld: ties the loaded registers to this point, so that
+// the compiler cannot move their uses above the wait (the load writes them
+// asynchronously).
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N])
+{
+    #pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
 {
     asm volatile(
