@@ -73,6 +73,14 @@ def kept_flops_from_mask(mask, wl) -> float:
     return float((4 * d * (cols * r[None, :]).sum()).item())
 
 
+# DRAM bytes (read + write) per (token, head) of one block_sparse_attn_kernel<128>
+# launch, from an ncu capture at 480p (395.2 MB / (32,760 tokens x 12 heads)).  The
+# kernel's DRAM traffic is its compulsory Q/K/V reads and O writes (K/V re-reads hit
+# L2), so it scales with the token-heads of the workload.  Re-measure whenever the
+# kernel changes.
+ATTN_DRAM_BYTES_PER_TOKEN_HEAD = 395.2e6 / (32760 * 12)
+
+
 def mask_bytes(wl, mask) -> float:
     """Algorithmic HBM bytes of mask prediction: Q and K read once + CSR written."""
     qk = 2 * wl.batch * wl.heads * wl.num_tokens * wl.head_dim * 2
@@ -95,6 +103,7 @@ class ClockSampler:
             sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
         except Exception:
             sel = []
+        self.sel = sel
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             self.fh = os.fdopen(fd, "w")
@@ -119,6 +128,17 @@ class ClockSampler:
                 if len(parts) >= 9:
                     rows.append(parts)
         os.unlink(self.path)
+        window = "timed region"
+        if not rows:
+            # The timed region was shorter than the sampler's start-up: one
+            # query right after it, under the same residency.
+            try:
+                out = subprocess.run(["nvidia-smi", *self.sel, f"--query-gpu={self.Q}", "--format=csv,noheader"],
+                                     capture_output=True, text=True, timeout=20).stdout
+                rows = [[p.strip() for p in l.split(",")] for l in out.splitlines() if l.count(",") >= 8]
+                window = "one sample right after the timed region (region shorter than the sampler start-up)"
+            except Exception:
+                rows = []
         if not rows:
             return None
 
@@ -133,7 +153,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(power)}
+                "power_w_max": max(power), "window": window}
 
 
 def combine_over_ranks(ms_step, attn_ms, e2e_ms, flops, dist=None, device="cpu"):
@@ -326,6 +346,10 @@ def main():
     Tb = wl.num_blocks
     density = kept_pairs / (wl.batch * wl.heads * Tb * Tb)
 
+    # Inputs smaller than twice the L2 (126 MB) would be timed warm: write a
+    # 256 MB buffer before every timed step and time the steps one by one.
+    resident = 4 * q.numel() * 2
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if resident < (252 << 20) else None
     sampler = ClockSampler(local_rank)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -334,13 +358,18 @@ def main():
     torch.cuda.synchronize()
     t_start.record(stream)
     for s in range(args.steps):
+        if flush is not None:
+            flush.fill_(s & 0xff)
         step(evs[s])
     t_end.record(stream)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     clocks = sampler.stop()
-    total_ms = t_start.elapsed_time(t_end)
+    if flush is None:
+        total_ms = t_start.elapsed_time(t_end)
+    else:
+        total_ms = sum(e[0].elapsed_time(e[5]) for e in evs)
     stage_ms = {name: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
                 for name, a, b in (("permute_qk_pool", 0, 1), ("permute_v", 1, 2), ("predict_mask_pooled", 2, 3),
                                    ("block_sparse_attn", 3, 4), ("unpermute", 4, 5))}
@@ -425,11 +454,14 @@ def main():
         "config": {"workload": workload_desc(wl), "global_batch": world * wl.batch, "seq_len": wl.num_tokens,
                    "parallelism": f"dp{world} (independent batch element per GPU, no collective)",
                    "kept_pairs_per_gpu": kept_pairs, "density": density,
-                   "l2": "inputs larger than L2 (774 MB per tensor), no flush"},
+                   "l2": (f"inputs larger than L2 ({q.numel() * 2 / 1e6:.0f} MB per tensor), no flush" if flush is None
+                          else "256 MB buffer written before every timed step; steps timed one by one")},
         "roofline": {"bound": "tensor", "kernel": "block_sparse_attn", "achieved": attn_tf,
                      "peak": attn_peak, "unit": "TFLOP/s", "frac": attn_tf / attn_peak,
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
-                     "traffic": None},
+                     "traffic": ATTN_DRAM_BYTES_PER_TOKEN_HEAD * wl.num_tokens * wl.batch * wl.heads,
+                     "traffic_source": "dram read+write of one ncu capture at 480p, scaled by token-heads "
+                                       "(profiles/attn_video480p_ncu.md)"},
         "stages": stages,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,

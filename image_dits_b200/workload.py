@@ -62,6 +62,9 @@ WORKLOADS = {
     "image": Workload("image", 1, 24, 128, 1, 64, 64, 1, 8, 8, 0.5, False, (0, 64, 64)),
     "video480p": Workload("video480p", 1, 12, 128, 21, 30, 52, 4, 4, 4, 0.2, True, (44, 42, 42)),
     "video720p": Workload("video720p", 1, 40, 128, 21, 45, 80, 4, 4, 4, 0.2, True, (44, 42, 42)),
+    # Qwen-image-edit shape (image, 60% sparsity): the latent size is not given, so the
+    # 64x64 image grid stands in, kept at 40% of the key blocks, 2D 8x8 windows, no sink.
+    "qwen_image": Workload("qwen_image", 1, 24, 128, 1, 64, 64, 1, 8, 8, 0.4, False, (0, 64, 64)),
 }
 SWEEP_KEEPS = (1.0, 0.5, 0.2, 0.1, 0.05)
 

@@ -72,8 +72,9 @@ def test_small_case_parity(name, wl):
     assert np.array_equal(bits(out["o"]), oracle.unpermute(bits(out["op"]), perm))
 
 
-def test_image_parity():
-    wl = WORKLOADS["image"]
+@pytest.mark.parametrize("name", ["image", "qwen_image"])
+def test_image_parity(name):
+    wl = WORKLOADS[name]
     q, k, v = make_qkv(wl, "cuda", seed=0)
     g = rf2.geometry_of(wl)
     out = run_path(g, q, k, v, wl.keep)
