@@ -57,6 +57,7 @@ def _load():
         lib.orc_block_means.argtypes = [vp, i64, i64, i64, vp]
         lib.orc_pooled_scores.argtypes = [vp, vp, i64, i64, i64, vp]
         lib.orc_select_blocks.argtypes = [vp, i64, i64, i64, i64, vp, vp]
+        lib.orc_select_cdf.argtypes = [vp, i64, i64, ctypes.c_double, i64, vp, vp, vp]
         lib.orc_masked_attention.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp, i64, vp, vp]
         lib.orc_num_threads.restype = i32
         _lib = lib
@@ -165,6 +166,36 @@ def select_blocks(S: np.ndarray, n: int, sink_first: int):
     thr = np.empty(S.shape[:-1], dtype=np.float64)
     _load().orc_select_blocks(_ptr(S), BH, Tb, n, sink_first, _ptr(mask), _ptr(thr))
     return mask, thr
+
+
+def select_cdf(S: np.ndarray, tau: float, sink_first: int):
+    """CDF-threshold selection plus the sink (section 2, online adaptive
+    patterns; section 3.4 for the sink).
+
+    Per non-sink row the key blocks in the order (score desc, j asc) are kept
+    until the cumulative softmax of the row's scores reaches tau.  Returns
+    (mask uint8 [..., T_b, T_b], cum float64 [..., T_b, 2], bnd float64
+    [..., T_b]): the cumulative probability before and after the last kept
+    block, and that block's score (NaN on sink rows)."""
+    S = np.ascontiguousarray(S, np.float64)
+    Tb = S.shape[-1]
+    BH = S.size // (Tb * Tb)
+    if not 0.0 < tau <= 1.0:
+        raise ValueError("tau out of range")
+    mask = np.empty(S.shape, dtype=np.uint8)
+    cum = np.empty(S.shape[:-1] + (2,), dtype=np.float64)
+    bnd = np.empty(S.shape[:-1], dtype=np.float64)
+    _load().orc_select_cdf(_ptr(S), BH, Tb, ctypes.c_double(tau), sink_first, _ptr(mask), _ptr(cum), _ptr(bnd))
+    return mask, cum, bnd
+
+
+def predict_mask_cdf(qp, kp, tau: float, T: int, H: int, W: int, sink: bool):
+    """Mask prediction with CDF-threshold selection: means, scores, CDF + sink.
+    Returns (mask, cum, bnd, S)."""
+    qm, km = block_means(qp), block_means(kp)
+    S = pooled_scores(qm, km)
+    mask, cum, bnd = select_cdf(S, tau, sink_start(T, H, W, sink))
+    return mask, cum, bnd, S
 
 
 def masked_attention(qp, kp, vp, mask: np.ndarray, items=None):

@@ -212,6 +212,63 @@ void orc_select_blocks(const double* S, int64_t BH, int64_t Tb, int64_t n, int64
     }
 }
 
+/*
+ * CDF-threshold selection ("RainFusion2.0" section 2, online adaptive
+ * patterns: the top blocks of the pooled-score attention are kept until
+ * their cumulative distribution reaches a threshold), with the sink of
+ * section 3.4 added as for top-n.
+ * Per non-sink row: p_j = exp(S_ij - max_j S_ij) / sum_j exp(...), the key
+ * blocks in the order (score desc, j asc), and the first m of them kept,
+ * m = the smallest count whose cumulative p reaches tau (tau in (0, 1]).
+ * Sink rows keep every column.
+ * cum[bh, i, 0] / cum[bh, i, 1] receive the cumulative p of the first m-1 and
+ * of the first m blocks (NaN for sink rows); bnd[bh, i] the score of the
+ * m-th block.
+ */
+void orc_select_cdf(const double* S, int64_t BH, int64_t Tb, double tau, int64_t sink_start,
+                    uint8_t* mask, double* cum, double* bnd)
+{
+    #pragma omp parallel
+    {
+        scored* buf = (scored*)malloc(sizeof(scored) * (size_t)Tb);
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t bh = 0; bh < BH; ++bh)
+            for (int64_t i = 0; i < Tb; ++i) {
+                const int64_t row = bh * Tb + i;
+                uint8_t* m = mask + row * Tb;
+                const double* s = S + row * Tb;
+                if (sink_start >= 0 && i >= sink_start) {
+                    for (int64_t j = 0; j < Tb; ++j) m[j] = 1;
+                    cum[2 * row] = NAN;
+                    cum[2 * row + 1] = NAN;
+                    bnd[row] = NAN;
+                    continue;
+                }
+                double mx = s[0];
+                for (int64_t j = 1; j < Tb; ++j) mx = s[j] > mx ? s[j] : mx;
+                double z = 0.0;
+                for (int64_t j = 0; j < Tb; ++j) z += exp(s[j] - mx);
+                for (int64_t j = 0; j < Tb; ++j) { buf[j].v = s[j]; buf[j].j = j; m[j] = 0; }
+                qsort(buf, (size_t)Tb, sizeof(scored), scored_cmp);
+                double c = 0.0, before = 0.0;
+                int64_t r = 0;
+                for (; r < Tb; ++r) {
+                    before = c;
+                    c += exp(buf[r].v - mx) / z;
+                    m[buf[r].j] = 1;
+                    if (c >= tau) break;
+                }
+                if (r == Tb) r = Tb - 1;               /* rounding kept the sum below tau */
+                cum[2 * row] = before;
+                cum[2 * row + 1] = c;
+                bnd[row] = buf[r].v;
+                if (sink_start >= 0)
+                    for (int64_t j = sink_start; j < Tb; ++j) m[j] = 1;
+            }
+        free(buf);
+    }
+}
+
 /* ------------------------------------------------------------------------- */
 /* Attention under a block mask (section 3.1): for every valid query row x of */
 /* block i, softmax(q_x K_J^T / sqrt(d)) V_J over the valid key rows of the   */

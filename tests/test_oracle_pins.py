@@ -246,3 +246,80 @@ def test_sink_rows_and_columns():
     assert mask[:, :, s0:].all()
     counts = mask[:, :s0].sum(-1)
     assert (counts >= 4).all() and (counts <= 4 + 4).all()
+
+
+# ---- CDF-threshold selection (section 2, online adaptive patterns) --------------------------
+
+
+def test_cdf_uniform_scores_closed_form():
+    """Equal scores: every block has p = 1/T_b, so m = ceil(tau * T_b) blocks,
+    and the tie rule keeps the lowest indices."""
+    Tb = 20
+    S = np.full((1, Tb, Tb), 0.37)
+    for tau, m in ((0.33, 7), (0.52, 11), (0.04, 1), (0.96, 20), (0.051, 2)):   # tau*T_b off the integers
+        mask, cum, bnd = oracle.select_cdf(S, tau, -1)
+        for i in range(Tb):
+            assert np.array_equal(np.nonzero(mask[0, i])[0], np.arange(m)), (tau, m)
+            assert cum[0, i, 1] >= tau > cum[0, i, 0]
+
+
+def test_cdf_two_levels_hand_computed():
+    """Three blocks with exp-weight 10, seventeen with weight 1 (total 47):
+    cumulative 10/47, 20/47, 30/47, then +1/47 per low block."""
+    Tb = 20
+    row = np.zeros(Tb)
+    hi = [4, 11, 17]
+    row[hi] = math.log(10.0)
+    S = row[None, None, :].repeat(Tb, 1)
+    # tau 0.5: 20/47 = 0.4255 < 0.5 <= 30/47 -> the three high blocks
+    mask, cum, _ = oracle.select_cdf(S, 0.5, -1)
+    assert np.array_equal(np.nonzero(mask[0, 0])[0], hi)
+    assert abs(cum[0, 0, 1] - 30 / 47) < 1e-12 and abs(cum[0, 0, 0] - 20 / 47) < 1e-12
+    # tau 0.7: 30/47 + k/47 >= 0.7 -> k = 3 low blocks, the lowest indices (0, 1, 2)
+    mask, cum, _ = oracle.select_cdf(S, 0.7, -1)
+    assert np.array_equal(np.nonzero(mask[0, 0])[0], sorted(hi + [0, 1, 2]))
+    assert abs(cum[0, 0, 1] - 33 / 47) < 1e-12
+    # tau tiny: the single best block (lowest j among the equal best)
+    mask, _, _ = oracle.select_cdf(S, 1e-9, -1)
+    assert np.array_equal(np.nonzero(mask[0, 0])[0], [4])
+
+
+def test_cdf_random_rows_brute_force():
+    """The kept set is the shortest prefix of the (score desc, j asc) order whose
+    softmax mass reaches tau (numpy lexsort + cumsum as the independent check)."""
+    rng = np.random.default_rng(5)
+    for Tb in (1, 2, 7, 33, 100):
+        S = rng.normal(0.0, 2.0, size=(2, Tb, Tb))
+        S[1, :, : Tb // 3] = S[1, :, :1]                   # ties
+        for tau in (0.1, 0.5, 0.9, 0.999):
+            mask, cum, bnd = oracle.select_cdf(S, tau, -1)
+            for bh in range(2):
+                for i in range(Tb):
+                    s = S[bh, i]
+                    order = np.lexsort((np.arange(Tb), -s))
+                    p = np.exp(s - s.max())
+                    p /= p.sum()
+                    c = np.cumsum(p[order])
+                    m = int(np.searchsorted(c >= tau, True)) + 1 if (c >= tau).any() else Tb
+                    want = np.zeros(Tb, np.uint8)
+                    want[order[:m]] = 1
+                    assert np.array_equal(mask[bh, i], want), (Tb, tau, bh, i)
+                    assert bnd[bh, i] == s[order[m - 1]]
+
+
+def test_cdf_tau_one_keeps_everything_and_sink():
+    rng = np.random.default_rng(6)
+    Tb = 24
+    S = rng.normal(size=(1, Tb, Tb))
+    mask, _, _ = oracle.select_cdf(S, 1.0, -1)
+    assert mask.all()
+    mask, cum, _ = oracle.select_cdf(S, 0.3, 20)
+    assert mask[0, 20:].all() and np.isnan(cum[0, 20:]).all()       # sink rows full
+    assert mask[0, :20, 20:].all()                                    # sink columns kept
+    # the CDF runs over every key block, sink columns included: where they carry the
+    # mass a row keeps no other block; otherwise its kept non-sink blocks are its best
+    s = S[0, :20]
+    for i in range(20):
+        kept = np.nonzero(mask[0, i, :20])[0]
+        if kept.size:
+            assert s[i, kept].min() >= np.sort(s[i, :20])[::-1][kept.size - 1]
