@@ -275,6 +275,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="video720p", choices=list(WORKLOADS))
     ap.add_argument("--keep", type=float, default=None)
+    ap.add_argument("--tau", type=float, default=None,
+                    help="CDF-threshold selection with this tau instead of the workload's top-n keep ratio")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="also time the keep-ratio sweep (stderr)")
@@ -309,7 +311,7 @@ def main():
     g = rf2.geometry_of(wl)
     q, k, v = make_qkv(wl, dev, seed=rank_seed(rank))
     qp, kp, vp, op, o = (torch.empty_like(q) for _ in range(5))
-    mask, ws = rf2.alloc_mask(g, wl.keep, dev)
+    mask, ws = rf2.alloc_mask(g, 1.0 if args.tau is not None else wl.keep, dev)
     stream = torch.cuda.current_stream()
 
     score_groups = -(-wl.batch * wl.heads // 16)
@@ -323,7 +325,10 @@ def main():
         rf2.permute(g, v, vp)
         if ev is not None:
             ev[2].record(stream)
-        rf2.predict_mask_pooled(g, wl.keep, mask, ws)
+        if args.tau is not None:
+            rf2.predict_mask_cdf_pooled(g, args.tau, mask, ws)
+        else:
+            rf2.predict_mask_pooled(g, wl.keep, mask, ws)
         if ev is not None:
             ev[3].record(stream)
         rf2.block_sparse_attn(g, qp, kp, vp, mask, op)
@@ -451,7 +456,10 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) + 0.5*smooth 3D field, 3D RoPE on Q/K, bf16)",
-        "config": {"workload": workload_desc(wl), "global_batch": world * wl.batch, "seq_len": wl.num_tokens,
+        "config": {"workload": workload_desc(wl) if args.tau is None else
+                   workload_desc(wl).split(", keep")[0] + f", CDF-threshold selection tau={args.tau:g} + first-frame "
+                   f"sink={'on' if wl.sink else 'off'}",
+                   "global_batch": world * wl.batch, "seq_len": wl.num_tokens,
                    "parallelism": f"dp{world} (independent batch element per GPU, no collective)",
                    "kept_pairs_per_gpu": kept_pairs, "density": density,
                    "l2": (f"inputs larger than L2 ({q.numel() * 2 / 1e6:.0f} MB per tensor), no flush" if flush is None
@@ -472,13 +480,15 @@ def main():
                        "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]}
 
     # mask prediction as one call on the permuted Q/K (Q and K read again), for its HBM roofline
+    predict = ((lambda: rf2.predict_mask_cdf(g, qp, kp, args.tau, mask, ws)) if args.tau is not None
+               else (lambda: rf2.predict_mask(g, qp, kp, wl.keep, mask, ws)))
     for _ in range(3):
-        rf2.predict_mask(g, qp, kp, wl.keep, mask, ws)
+        predict()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(5):
-        rf2.predict_mask(g, qp, kp, wl.keep, mask, ws)
+        predict()
     b.record(stream)
     torch.cuda.synchronize()
     ms_pm = a.elapsed_time(b) / 5

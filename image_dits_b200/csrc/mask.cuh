@@ -16,6 +16,7 @@
 //                     (equal scores: lower j), union the sink columns, and
 //                     write the row as an ascending CSR list.  Sink rows keep
 //                     every column.
+// select_cdf_kernel   the CDF-threshold alternative to top-n (see below).
 #pragma once
 #include "geometry.cuh"
 #include "ptx.cuh"
@@ -499,6 +500,123 @@ __global__ void __launch_bounds__(kSelThreads) select_from_scores_kernel(const f
     uint32_t* hist = hist_all + warp * 256;
     for (int r = warp; r < nrows; r += kSelThreads / 32)
         select_row(keys + (size_t)r * Tb, hist, mg, bh, i0 + r, lane, row_start, row_count, col_idx, keep_all);
+}
+
+// CDF-threshold selection ("RainFusion2.0" section 2, online adaptive
+// patterns: the best key blocks of a row are kept until the cumulative
+// softmax of its pooled scores reaches tau), the sink of section 3.4 added on
+// top.  One warp per row, the row's order keys and weights in shared memory:
+//   w_j = 2^((S_j - max) log2 e)  and  Z = sum_j w_j  (fp32; each lane sums its
+//   columns in ascending order, then an xor butterfly, so every lane holds the
+//   same bits),
+//   K* = the largest key with W(>= K*) >= tau Z, found by bisection over the
+//   row's key range (W(>= K) summed the same way),
+//   kept = {key > K*} plus the first c blocks of key K* in ascending j, c the
+//   smallest count with W(> K*) + c w(K*) >= tau Z.
+// This is the shortest prefix of the (score desc, j asc) order whose mass
+// reaches tau.  Rows use the full capacity T_b (make_mask_geo with
+// n_keep = T_b), so row offsets stay closed-form.
+__device__ __forceinline__ float warp_sum_same(float v)
+{
+    #pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+template <int R>
+__global__ void __launch_bounds__(32 * R) select_cdf_kernel(const float* __restrict__ S, int32_t ld_s,
+                                                            int32_t* __restrict__ row_start,
+                                                            int32_t* __restrict__ row_count,
+                                                            int32_t* __restrict__ col_idx, MaskGeo mg, int64_t h0,
+                                                            float tau)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const int Tb = mg.Tb;
+    const int lane = threadIdx.x & 31;
+    const int r = threadIdx.x >> 5;
+    const int64_t hl = blockIdx.y;
+    const int64_t bh = h0 + hl;
+    const int i = blockIdx.x * R + r;
+    if (i >= Tb) return;                                   // whole warp
+    uint32_t* key = reinterpret_cast<uint32_t*>(smem_raw) + (size_t)r * Tb;
+    float* w = reinterpret_cast<float*>(smem_raw) + (size_t)R * Tb + (size_t)r * Tb;
+    const int64_t rs = row_offset(mg, bh, i);
+    const int64_t row_id = bh * Tb + i;
+    int32_t* out = col_idx + rs;
+    if (i >= mg.sink_first) {
+        for (int j = lane; j < Tb; j += 32) out[j] = j;
+        if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = Tb; }
+        return;
+    }
+    const float* src = S + (hl * Tb + i) * (int64_t)ld_s;
+    float mx = -INFINITY;
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int j = lane; j < Tb; j += 32) {
+        const float v = src[j];
+        const uint32_t k = float_order_key(v);
+        key[j] = k;
+        mx = fmaxf(mx, v);
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+    }
+    #pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    float z = 0.f;
+    for (int j = lane; j < Tb; j += 32) {
+        const float v = src[j];
+        const float wj = exp2f((v - mx) * 1.4426950408889634f);
+        w[j] = wj;
+        z += wj;
+    }
+    z = warp_sum_same(z);
+    const float target = tau * z;
+    __syncwarp();
+    auto mass_ge = [&](uint32_t K) -> float {
+        float a = 0.f;
+        for (int j = lane; j < Tb; j += 32) a += (key[j] >= K) ? w[j] : 0.f;
+        return warp_sum_same(a);
+    };
+    uint32_t lo = kmin, hi = kmax;                         // mass_ge(kmin) = z >= target
+    while (lo < hi) {
+        const uint32_t mid = lo + (uint32_t)(((uint64_t)hi - lo + 1) >> 1);
+        if (mass_ge(mid) >= target) lo = mid;
+        else hi = mid - 1;
+    }
+    const uint32_t thr = lo;
+    const float w_gt = (thr == 0xffffffffu) ? 0.f : mass_ge(thr + 1);
+    int n_eq = 0;
+    float w_eq = 0.f;
+    for (int j0 = 0; j0 < Tb; j0 += 32) {
+        const int j = j0 + lane;
+        const bool eq = (j < Tb) && key[j] == thr;
+        const uint32_t b = __ballot_sync(0xffffffffu, eq);
+        if (b && w_eq == 0.f) w_eq = __shfl_sync(0xffffffffu, eq ? w[j] : 0.f, __ffs(b) - 1);
+        n_eq += __popc(b);
+    }
+    int c = 1;
+    if (n_eq > 1 && w_eq > 0.f) {
+        c = (int)ceilf((target - w_gt) / w_eq);
+        c = max(1, min(n_eq, c));
+        while (c > 1 && w_gt + (float)(c - 1) * w_eq >= target) --c;
+        while (c < n_eq && w_gt + (float)c * w_eq < target) ++c;
+    }
+    int eq_left = c;
+    int written = 0;
+    for (int j0 = 0; j0 < Tb; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t k = (j < Tb) ? key[j] : 0u;
+        const bool eq = (j < Tb) && (k == thr);
+        const uint32_t eq_ballot = __ballot_sync(0xffffffffu, eq);
+        const int eq_rank = __popc(eq_ballot & ((1u << lane) - 1u));
+        const bool sel = (j < Tb) && (k > thr || (eq && eq_rank < eq_left) || j >= mg.sink_first);
+        eq_left -= __popc(eq_ballot);
+        const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[written + __popc(sel_ballot & ((1u << lane) - 1u))] = j;
+        written += __popc(sel_ballot);
+    }
+    if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = written; }
 }
 
 }  // namespace rf2

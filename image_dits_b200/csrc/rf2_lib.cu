@@ -299,6 +299,21 @@ static int launch_select(const Checked& c, const MaskGeo& mg, const float* S, in
     return launch_status();
 }
 
+// CDF-threshold selection for a group of heads: one warp per row, R rows per
+// CTA, the rows' keys and weights in shared memory (R * T_b * 8 bytes).
+template <int R>
+static int launch_select_cdf(const Checked& c, const MaskGeo& mg, const float* S, int64_t h0, int64_t g,
+                             int32_t* row_start, int32_t* row_count, int32_t* col_idx, float tau, cudaStream_t s)
+{
+    const size_t smem = (size_t)R * c.Tb * 8;
+    if (cudaFuncSetAttribute(select_cdf_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return RF2_ERR_CUDA;
+    dim3 grid((c.Tb + R - 1) / R, (unsigned)g);
+    select_cdf_kernel<R><<<grid, 32 * R, smem, s>>>(S, score_ld(c.Tb), row_start, row_count, col_idx, mg, h0, tau);
+    return launch_status();
+}
+
 // Block means, then per group of heads the tensor-core scores and the
 // selection.  `ws` holds the means followed by a score buffer for as many
 // heads (at most kScoreGroupHeads) as `ws_bytes` allows.
@@ -323,9 +338,10 @@ static int mask_ws(const Checked& c, void* ws, size_t ws_bytes, MaskWs* w)
     return RF2_OK;
 }
 
-// Per group of heads: the tensor-core scores, then the selection.
+// Per group of heads: the tensor-core scores, then the selection (top-n, or
+// the CDF threshold when tau > 0).
 static int launch_score_select(const Checked& c, const MaskGeo& mg, const MaskWs& w, int32_t* row_start,
-                               int32_t* row_count, int32_t* col_idx, cudaStream_t s)
+                               int32_t* row_count, int32_t* col_idx, cudaStream_t s, float tau = 0.f)
 {
     int r = RF2_OK;
     for (int64_t h0 = 0; r == RF2_OK && h0 < c.BH; h0 += w.G) {
@@ -333,14 +349,19 @@ static int launch_score_select(const Checked& c, const MaskGeo& mg, const MaskWs
         r = (c.D == 128) ? launch_scores<128>(c, w.means_hi, w.means_lo, w.S, h0, g, s)
                          : launch_scores<64>(c, w.means_hi, w.means_lo, w.S, h0, g, s);
         if (r != RF2_OK) break;
-        r = launch_select<8>(c, mg, w.S, h0, g, row_start, row_count, col_idx, s);
+        if (tau > 0.f)
+            r = (c.Tb <= 1600) ? launch_select_cdf<8>(c, mg, w.S, h0, g, row_start, row_count, col_idx, tau, s)
+                               : launch_select_cdf<4>(c, mg, w.S, h0, g, row_start, row_count, col_idx, tau, s);
+        else
+            r = launch_select<8>(c, mg, w.S, h0, g, row_start, row_count, col_idx, s);
     }
     return r;
 }
 
 // Block means of the permuted Q and K, then scores and selection.
 static int launch_mask(const Checked& c, const MaskGeo& mg, const void* qp, const void* kp, int32_t* row_start,
-                       int32_t* row_count, int32_t* col_idx, void* ws, size_t ws_bytes, cudaStream_t s)
+                       int32_t* row_count, int32_t* col_idx, void* ws, size_t ws_bytes, cudaStream_t s,
+                       float tau = 0.f)
 {
     MaskWs w;
     const int st = mask_ws(c, ws, ws_bytes, &w);
@@ -357,7 +378,7 @@ static int launch_mask(const Checked& c, const MaskGeo& mg, const void* qp, cons
                                                     c.N, c.Tb, c.BH);
     const int r = launch_status();
     if (r != RF2_OK) return r;
-    return launch_score_select(c, mg, w, row_start, row_count, col_idx, s);
+    return launch_score_select(c, mg, w, row_start, row_count, col_idx, s, tau);
 }
 
 // ------------------------------------------------------------------------
@@ -537,6 +558,46 @@ int rf2_predict_mask_pooled(const rf2_geometry* geom, double keep_ratio, int32_t
     const int ws_st = mask_ws(c, workspace, workspace_bytes, &w);
     if (ws_st != RF2_OK) return ws_st;
     return launch_score_select(c, mg, w, row_start, row_count, col_idx, reinterpret_cast<cudaStream_t>(stream));
+}
+
+static bool tau_ok(double tau) { return tau > 0.0 && tau <= 1.0; }
+
+int rf2_predict_mask_cdf(const rf2_geometry* geom, const void* qp, const void* kp, double tau, int32_t* row_start,
+                         int32_t* row_count, int32_t* col_idx, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Checked c;
+    MaskGeo mg;
+    rf2_sizes sz;
+    const int st = sizes_for(geom, 1.0, c, mg, &sz);      // rows at full capacity T_b
+    if (st != RF2_OK) return st;
+    if (!tau_ok(tau)) return RF2_ERR_INVALID_ARGUMENT;
+    if (!qp || !kp || !row_start || !row_count || !col_idx || !workspace) return RF2_ERR_INVALID_ARGUMENT;
+    if (!aligned16(qp) || !aligned16(kp) || !aligned16(workspace) || !aligned16(row_start) || !aligned16(row_count) ||
+        !aligned16(col_idx))
+        return RF2_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < sz.mask_workspace_bytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    return launch_mask(c, mg, qp, kp, row_start, row_count, col_idx, workspace, workspace_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), (float)tau);
+}
+
+int rf2_predict_mask_cdf_pooled(const rf2_geometry* geom, double tau, int32_t* row_start, int32_t* row_count,
+                                int32_t* col_idx, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Checked c;
+    MaskGeo mg;
+    rf2_sizes sz;
+    const int st = sizes_for(geom, 1.0, c, mg, &sz);
+    if (st != RF2_OK) return st;
+    if (!tau_ok(tau)) return RF2_ERR_INVALID_ARGUMENT;
+    if (!row_start || !row_count || !col_idx || !workspace) return RF2_ERR_INVALID_ARGUMENT;
+    if (!aligned16(workspace) || !aligned16(row_start) || !aligned16(row_count) || !aligned16(col_idx))
+        return RF2_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < sz.mask_workspace_bytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    MaskWs w;
+    const int ws_st = mask_ws(c, workspace, workspace_bytes, &w);
+    if (ws_st != RF2_OK) return ws_st;
+    return launch_score_select(c, mg, w, row_start, row_count, col_idx, reinterpret_cast<cudaStream_t>(stream),
+                               (float)tau);
 }
 
 int rf2_device_status(void* stream)

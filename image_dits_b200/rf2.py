@@ -27,6 +27,7 @@ RF2_ERR_TIMEOUT = 5
 EXPORTED = (
     "rf2_status_string", "rf2_query", "rf2_permutation_index", "rf2_permute", "rf2_unpermute",
     "rf2_predict_mask", "rf2_predict_mask_static", "rf2_permute_qk_pool", "rf2_predict_mask_pooled",
+    "rf2_predict_mask_cdf", "rf2_predict_mask_cdf_pooled",
     "rf2_block_sparse_attn", "rf2_device_status",
 )
 
@@ -78,6 +79,8 @@ def lib():
         L.rf2_predict_mask_static.argtypes = [G, vp, vp, f64, vp, vp, vp, vp]
         L.rf2_permute_qk_pool.argtypes = [G, vp, vp, vp, vp, vp, sz, vp]
         L.rf2_predict_mask_pooled.argtypes = [G, f64, vp, vp, vp, vp, sz, vp]
+        L.rf2_predict_mask_cdf.argtypes = [G, vp, vp, f64, vp, vp, vp, vp, sz, vp]
+        L.rf2_predict_mask_cdf_pooled.argtypes = [G, f64, vp, vp, vp, vp, sz, vp]
         L.rf2_block_sparse_attn.argtypes = [G, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.rf2_device_status.argtypes = [vp]
         for name in EXPORTED:
@@ -193,6 +196,31 @@ def predict_mask(geom: Geometry, qp: torch.Tensor, kp: torch.Tensor, keep: float
                                   mask.row_start.data_ptr(), mask.row_count.data_ptr(), mask.col_idx.data_ptr(),
                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                   _stream(stream)), "rf2_predict_mask")
+    return mask
+
+
+def predict_mask_cdf(geom: Geometry, qp: torch.Tensor, kp: torch.Tensor, tau: float, mask: BlockMask | None = None,
+                     workspace: torch.Tensor | None = None, stream=None) -> BlockMask:
+    """CDF-threshold mask (rows sized at full capacity: alloc_mask(geom, 1.0, ...))."""
+    _check_qkv(geom, qp, kp)
+    if mask is None or workspace is None:
+        m2, ws2 = alloc_mask(geom, 1.0, qp.device)
+        mask = mask or m2
+        workspace = ws2 if workspace is None else workspace
+    _check(lib().rf2_predict_mask_cdf(ctypes.byref(geom), qp.data_ptr(), kp.data_ptr(), float(tau),
+                                      mask.row_start.data_ptr(), mask.row_count.data_ptr(), mask.col_idx.data_ptr(),
+                                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                      _stream(stream)), "rf2_predict_mask_cdf")
+    return mask
+
+
+def predict_mask_cdf_pooled(geom: Geometry, tau: float, mask: BlockMask, workspace: torch.Tensor,
+                            stream=None) -> BlockMask:
+    """CDF-threshold mask from the block means rf2_permute_qk_pool left in `workspace`."""
+    _check(lib().rf2_predict_mask_cdf_pooled(ctypes.byref(geom), float(tau), mask.row_start.data_ptr(),
+                                             mask.row_count.data_ptr(), mask.col_idx.data_ptr(),
+                                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                             _stream(stream)), "rf2_predict_mask_cdf_pooled")
     return mask
 
 

@@ -160,6 +160,28 @@ int rf2_permute_qk_pool(const rf2_geometry* geom, const void* q_bf16, const void
 int rf2_predict_mask_pooled(const rf2_geometry* geom, double keep_ratio, int32_t* row_start, int32_t* row_count,
                             int32_t* col_idx, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Mask prediction with CDF-threshold selection instead of a fixed top-n: the
+ * alternative the pages name among the online adaptive patterns (section 2,
+ * "Related Work" (2): block means -> scores -> the top blocks whose
+ * cumulative distribution meets a threshold).  Per non-sink query-block row,
+ * the pooled scores (eqs. (5)-(7)) are turned into p_j = softmax_j(S_ij); the
+ * key blocks are ordered by (score desc, j asc) and the shortest prefix whose
+ * cumulative p reaches tau (0 < tau <= 1) is kept; the first-frame sink is
+ * added as in rf2_predict_mask (section 3.4).  Rows are adaptive: every row
+ * has capacity T_b, so size the outputs with rf2_query(geom, 1.0, ...)
+ * (col_idx_capacity = B*H*T_b^2, row_start[r] = r*T_b); the workspace is
+ * mask_workspace_bytes of the same query.  Arithmetic is fp32 (weights
+ * 2^((S - max) log2 e), sums in a fixed order, so the result is
+ * deterministic).  tau outside (0, 1] -> RF2_ERR_INVALID_ARGUMENT; other
+ * errors as rf2_predict_mask. */
+int rf2_predict_mask_cdf(const rf2_geometry* geom, const void* qp_bf16, const void* kp_bf16, double tau,
+                         int32_t* row_start, int32_t* row_count, int32_t* col_idx, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* The same from the block means rf2_permute_qk_pool left in `workspace`. */
+int rf2_predict_mask_cdf_pooled(const rf2_geometry* geom, double tau, int32_t* row_start, int32_t* row_count,
+                                int32_t* col_idx, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Block-sparse FlashAttention forward (section 3.1): for every query block i,
  * O_i = softmax(Q_i K_J^T / sqrt(d)) V_J over the key blocks J kept in row i
  * of the CSR mask (eqs. (1)-(4); Q_i K_j^T and P_ij V_j are skipped when

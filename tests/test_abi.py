@@ -145,6 +145,20 @@ def test_host_validation(L):
         rf2.RF2_ERR_INVALID_ARGUMENT
     assert L.rf2_predict_mask_pooled(G(good), 0.5, fake, fake, fake, None, big, None) == \
         rf2.RF2_ERR_INVALID_ARGUMENT
+    # predict_mask_cdf / predict_mask_cdf_pooled: tau in (0, 1], workspace of rf2_query(geom, 1.0)
+    for tau in (0.0, -0.5, 1.5, float("nan")):
+        assert L.rf2_predict_mask_cdf(G(good), fake, fake, tau, fake, fake, fake, fake, big, None) == \
+            rf2.RF2_ERR_INVALID_ARGUMENT
+        assert L.rf2_predict_mask_cdf_pooled(G(good), tau, fake, fake, fake, fake, big, None) == \
+            rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_predict_mask_cdf(G(good), fake, fake, 0.5, fake, fake, fake, fake, ws_small, None) == \
+        rf2.RF2_ERR_INSUFFICIENT_WORKSPACE
+    assert L.rf2_predict_mask_cdf(G(good), None, fake, 0.5, fake, fake, fake, fake, big, None) == \
+        rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_predict_mask_cdf_pooled(G(good), 0.5, fake, fake, None, fake, big, None) == \
+        rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_predict_mask_cdf_pooled(G(bad_dim), 0.5, fake, fake, fake, fake, big, None) == \
+        rf2.RF2_ERR_UNSUPPORTED
     # block_sparse_attn
     assert L.rf2_block_sparse_attn(G(good), fake, fake, None, fake, fake, fake, fake, None, None) == \
         rf2.RF2_ERR_INVALID_ARGUMENT
