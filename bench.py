@@ -53,7 +53,7 @@ def load_peaks():
 
 def workload_desc(wl):
     return (f"{wl.name}: B={wl.batch}/GPU, {wl.heads} heads, d={wl.head_dim}, latent {wl.frames}x{wl.height}x"
-            f"{wl.width} ({wl.num_tokens:,} tokens), block 64, window {wl.win_t}x{wl.win_h}x{wl.win_w}, keep "
+            f"{wl.width}{f' + {wl.text_tokens} text' if wl.text_tokens else ''} ({wl.num_tokens:,} tokens), block 64, window {wl.win_t}x{wl.win_h}x{wl.win_w}, keep "
             f"{wl.keep:g} of key blocks (sparsity {1 - wl.keep:g}) + first-frame sink={'on' if wl.sink else 'off'}")
 
 
@@ -196,19 +196,19 @@ def oracle_sample(wl, seed=0, n_query_blocks=32, budget_s=None):
     import oracle
     from image_dits_b200.workload import Workload
     one = Workload(wl.name, 1, 1, wl.head_dim, wl.frames, wl.height, wl.width, wl.win_t, wl.win_h, wl.win_w,
-                   wl.keep, wl.sink, wl.rope)
+                   wl.keep, wl.sink, wl.rope, wl.text_tokens)
     q, k, v = make_qkv(one, "cpu", seed=seed)
 
     def bits(t):
         return t.contiguous().view(torch.int16).numpy().view(np.uint16)
     qb, kb, vb = bits(q), bits(k), bits(v)
     t0 = time.perf_counter()
-    perm = oracle.permutation(wl.frames, wl.height, wl.width, wl.win_t, wl.win_h, wl.win_w, wl.sink)
+    perm = oracle.permutation(wl.frames, wl.height, wl.width, wl.win_t, wl.win_h, wl.win_w, wl.sink, wl.text_tokens)
     qp, kp, vp = oracle.permute(qb, perm), oracle.permute(kb, perm), oracle.permute(vb, perm)
-    mask, _, _ = oracle.predict_mask(qp, kp, wl.keep, wl.frames, wl.height, wl.width, wl.sink)
+    mask, _, _ = oracle.predict_mask(qp, kp, wl.keep, wl.frames, wl.height, wl.width, wl.sink, wl.text_tokens)
     Tb = wl.num_blocks
     rng = np.random.default_rng(seed)
-    s0 = oracle.sink_start(wl.frames, wl.height, wl.width, wl.sink)
+    s0 = oracle.sink_start(wl.frames, wl.height, wl.width, wl.sink, wl.text_tokens)
     upper = s0 if s0 > 0 else Tb
     order = [int(i) for i in rng.permutation(upper) if i != Tb - 1]
     N = wl.num_tokens

@@ -2,9 +2,11 @@
 // row layout.  Used by host validation, rf2_permutation_index and the kernels.
 //
 // Window permutation ("RainFusion2.0", section 3.3 and section 1 Key Idea 2;
-// first frame moved to the end, section 3.4).  The sequence is one segment
+// first frame moved to the end, section 3.4).  The video part is one segment
 // (frames 0..F-1), or, with the first-frame sink on and F > 1, two: frames
-// 1..F-1 followed by frame 0.  Each segment is tiled from its origin by
+// 1..F-1 followed by frame 0.  Text tokens of a joint video-text attention
+// (section 3.4: the first frame is moved next to them) follow the video
+// tokens in the input and keep their place after the permuted video.  Each segment is tiled from its origin by
 // windows of (wt, wh, ww) frames/rows/columns, cut short at the grid edge.
 // Windows go in raster order and so do the tokens inside each window.
 // Because every window before the last one along an axis is full-sized, the
@@ -30,26 +32,29 @@ struct PermGeo {
     int32_t wt, wh, ww;    // window
     int32_t move_first;    // frame 0 moved behind frames 1..T-1
     int32_t HW;
-    int32_t N;
+    int32_t Nv;            // video tokens T*H*W
+    int32_t N;             // Nv + text tokens
 };
 
 RF2_HD int32_t imin(int32_t a, int32_t b) { return a < b ? a : b; }
 
 RF2_HD PermGeo make_perm_geo(int32_t T, int32_t H, int32_t W, int32_t wt, int32_t wh, int32_t ww,
-                             int32_t sink)
+                             int32_t sink, int32_t text)
 {
     PermGeo g;
     g.T = T; g.H = H; g.W = W; g.wt = wt; g.wh = wh; g.ww = ww;
     g.move_first = (sink && T > 1) ? 1 : 0;
     g.HW = H * W;
-    g.N = T * H * W;
+    g.Nv = T * H * W;
+    g.N = g.Nv + text;
     return g;
 }
 
 // Permuted position -> original raster index.
 RF2_HD int32_t perm_src(const PermGeo& g, int32_t p)
 {
-    const int32_t seg0 = g.move_first ? (g.T - 1) * g.HW : g.N;
+    if (p >= g.Nv) return p;                               // text tokens
+    const int32_t seg0 = g.move_first ? (g.T - 1) * g.HW : g.Nv;
     int32_t t0, F, q;
     if (p < seg0) { t0 = g.move_first; F = g.move_first ? g.T - 1 : g.T; q = p; }
     else          { t0 = 0;            F = 1;                          q = p - seg0; }
@@ -74,6 +79,7 @@ RF2_HD int32_t perm_src(const PermGeo& g, int32_t p)
 // Original raster index -> permuted position (inverse of perm_src).
 RF2_HD int32_t perm_dst(const PermGeo& g, int32_t s)
 {
+    if (s >= g.Nv) return s;                               // text tokens
     const int32_t t = s / g.HW;
     const int32_t hw = s - t * g.HW;
     const int32_t h = hw / g.W;
@@ -106,12 +112,21 @@ struct MaskGeo {
     int64_t head_total;  // col_idx slots per (b, h)
 };
 
-RF2_HD MaskGeo make_mask_geo(int32_t N, int32_t n_keep, int32_t sink_on, int32_t T, int32_t HW)
+// First token of the full-attention region of the permuted sequence: frame 0
+// (at the end of the video part) when the first-frame sink is on, else the
+// first text token; -1 when there is neither.
+RF2_HD int32_t sink_first_token(const PermGeo& g, int32_t sink_on)
+{
+    if (sink_on) return (g.T - 1) * g.HW;
+    return (g.N > g.Nv) ? g.Nv : -1;
+}
+
+RF2_HD MaskGeo make_mask_geo(int32_t N, int32_t n_keep, int32_t first_sink_token)
 {
     MaskGeo m;
     m.Tb = (N + kBlock - 1) / kBlock;
     m.n_keep = n_keep;
-    m.sink_first = sink_on ? ((T - 1) * HW) / kBlock : m.Tb;
+    m.sink_first = (first_sink_token >= 0) ? first_sink_token / kBlock : m.Tb;
     const int32_t n_sink = m.Tb - m.sink_first;
     m.cap = imin(m.Tb, n_keep + n_sink);
     m.head_total = (int64_t)m.sink_first * m.cap + (int64_t)n_sink * m.Tb;

@@ -43,9 +43,9 @@ static Checked check_geometry(const rf2_geometry* g)
     if (!g) return c;
     if (g->batch <= 0 || g->heads <= 0 || g->frames <= 0 || g->height <= 0 || g->width <= 0 ||
         g->win_t <= 0 || g->win_h <= 0 || g->win_w <= 0 || g->head_dim <= 0 || g->block <= 0 ||
-        (g->first_frame_sink != 0 && g->first_frame_sink != 1))
+        (g->first_frame_sink != 0 && g->first_frame_sink != 1) || g->text_tokens < 0)
         return c;
-    const int64_t N = (int64_t)g->frames * g->height * g->width;
+    const int64_t N = (int64_t)g->frames * g->height * g->width + g->text_tokens;
     if (N > INT32_MAX) return c;
     c.status = RF2_ERR_UNSUPPORTED;
     if (g->head_dim != 64 && g->head_dim != 128) return c;
@@ -58,7 +58,8 @@ static Checked check_geometry(const rf2_geometry* g)
     c.N = (int32_t)N;
     c.Tb = (int32_t)Tb;
     c.D = g->head_dim;
-    c.pg = make_perm_geo(g->frames, g->height, g->width, g->win_t, g->win_h, g->win_w, g->first_frame_sink);
+    c.pg = make_perm_geo(g->frames, g->height, g->width, g->win_t, g->win_h, g->win_w, g->first_frame_sink,
+                         g->text_tokens);
     c.status = RF2_OK;
     return c;
 }
@@ -91,7 +92,7 @@ static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg
     int32_t n = 0;
     const int st = keep_count(keep, c.Tb, &n);
     if (st != RF2_OK) return st;
-    mg = make_mask_geo(c.N, n, g->first_frame_sink, g->frames, g->height * g->width);
+    mg = make_mask_geo(c.N, n, sink_first_token(c.pg, g->first_frame_sink));
     const int64_t total = c.BH * mg.head_total;
     if (total > INT32_MAX) return RF2_ERR_UNSUPPORTED;
     if (out) {
@@ -478,7 +479,7 @@ int rf2_block_sparse_attn(const rf2_geometry* geom, const void* qp, const void* 
 {
     const Checked c = check_geometry(geom);
     if (c.status != RF2_OK) return c.status;
-    const MaskGeo mg = make_mask_geo(c.N, 1, geom->first_frame_sink, geom->frames, geom->height * geom->width);
+    const MaskGeo mg = make_mask_geo(c.N, 1, sink_first_token(c.pg, geom->first_frame_sink));
     if (!qp || !kp || !vp || !row_start || !row_count || !col_idx || !op) return RF2_ERR_INVALID_ARGUMENT;
     if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(op) || !aligned16(row_start) ||
         !aligned16(row_count) || !aligned16(col_idx) || (lse && !aligned16(lse)))

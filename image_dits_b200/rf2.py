@@ -35,7 +35,7 @@ EXPORTED = (
 class Geometry(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "heads", "head_dim", "frames", "height", "width",
-        "win_t", "win_h", "win_w", "block", "first_frame_sink")]
+        "win_t", "win_h", "win_w", "block", "first_frame_sink", "text_tokens")]
 
 
 class Sizes(ctypes.Structure):
@@ -99,14 +99,21 @@ def _check(status: int, what: str):
         raise Rf2Error(status, what)
 
 
-def make_geometry(batch, heads, head_dim, frames, height, width, win_t, win_h, win_w, sink, block=64) -> Geometry:
-    return Geometry(batch, heads, head_dim, frames, height, width, win_t, win_h, win_w, block, int(bool(sink)))
+def make_geometry(batch, heads, head_dim, frames, height, width, win_t, win_h, win_w, sink, block=64,
+                  text=0) -> Geometry:
+    return Geometry(batch, heads, head_dim, frames, height, width, win_t, win_h, win_w, block, int(bool(sink)),
+                    int(text))
+
+
+def num_tokens(geom: Geometry) -> int:
+    """Sequence length N: video tokens, then text tokens."""
+    return geom.frames * geom.height * geom.width + geom.text_tokens
 
 
 def geometry_of(wl, batch: int | None = None) -> Geometry:
     """Geometry of a ``workload.Workload``."""
     return make_geometry(wl.batch if batch is None else batch, wl.heads, wl.head_dim, wl.frames, wl.height,
-                         wl.width, wl.win_t, wl.win_h, wl.win_w, wl.sink)
+                         wl.width, wl.win_t, wl.win_h, wl.win_w, wl.sink, text=wl.text_tokens)
 
 
 def query(geom: Geometry, keep: float = 1.0) -> Sizes:
@@ -116,8 +123,7 @@ def query(geom: Geometry, keep: float = 1.0) -> Sizes:
 
 
 def permutation_index(geom: Geometry) -> np.ndarray:
-    n = geom.frames * geom.height * geom.width
-    perm = np.empty(n, dtype=np.int32)
+    perm = np.empty(num_tokens(geom), dtype=np.int32)
     _check(lib().rf2_permutation_index(ctypes.byref(geom), perm.ctypes.data), "rf2_permutation_index")
     return perm
 
@@ -129,7 +135,7 @@ def _stream(stream) -> int:
 
 
 def _check_qkv(geom: Geometry, *ts):
-    shape = (geom.batch, geom.heads, geom.frames * geom.height * geom.width, geom.head_dim)
+    shape = (geom.batch, geom.heads, num_tokens(geom), geom.head_dim)
     for t in ts:
         if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and tuple(t.shape) == shape):
             raise ValueError(f"expected a contiguous CUDA bf16 tensor of shape {shape}, got "
@@ -253,7 +259,7 @@ def block_sparse_attn(geom: Geometry, qp, kp, vp, mask: BlockMask, out: torch.Te
     out = torch.empty_like(qp) if out is None else out
     _check_qkv(geom, out)
     if lse is not None:
-        n = geom.frames * geom.height * geom.width
+        n = num_tokens(geom)
         if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
                 and lse.numel() == geom.batch * geom.heads * n):
             raise ValueError("lse must be a contiguous CUDA float32 tensor of B*H*N elements")

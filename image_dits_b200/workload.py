@@ -41,10 +41,15 @@ class Workload:
     keep: float
     sink: bool
     rope: tuple  # (t, h, w) channel split; t = 0 for images
+    text_tokens: int = 0  # joint-attention text tokens, stored after the video tokens
+
+    @property
+    def num_video_tokens(self) -> int:
+        return self.frames * self.height * self.width
 
     @property
     def num_tokens(self) -> int:
-        return self.frames * self.height * self.width
+        return self.num_video_tokens + self.text_tokens
 
     @property
     def num_blocks(self) -> int:
@@ -65,6 +70,9 @@ WORKLOADS = {
     # Qwen-image-edit shape (image, 60% sparsity): the latent size is not given, so the
     # 64x64 image grid stands in, kept at 40% of the key blocks, 2D 8x8 windows, no sink.
     "qwen_image": Workload("qwen_image", 1, 24, 128, 1, 64, 64, 1, 8, 8, 0.4, False, (0, 64, 64)),
+    # A video DiT with joint video-text attention: 256 text tokens after the 480p latent,
+    # grouped with the first frame into the full-attention region.
+    "video480p_text": Workload("video480p_text", 1, 12, 128, 21, 30, 52, 4, 4, 4, 0.2, True, (44, 42, 42), 256),
 }
 SWEEP_KEEPS = (1.0, 0.5, 0.2, 0.1, 0.05)
 
@@ -109,7 +117,9 @@ def _rope_(x: torch.Tensor, wl: Workload, theta: float = 10000.0) -> None:
 
 
 def make_qkv(wl: Workload, device="cpu", seed: int = 0, batch: int | None = None):
-    """Return (q, k, v) bf16 [B, heads, N, d] on `device`, in [F,H,W] order."""
+    """Return (q, k, v) bf16 [B, heads, N, d] on `device`: the video tokens in
+    [F,H,W] order (field + noise, RoPE on Q and K), then the text tokens (noise
+    only, no positional rotation)."""
     B = wl.batch if batch is None else batch
     g = torch.Generator(device=device)
     g.manual_seed(seed)
@@ -120,9 +130,10 @@ def make_qkv(wl: Workload, device="cpu", seed: int = 0, batch: int | None = None
         gi.manual_seed(seed + 1 + idx)
         x = torch.randn((B, wl.heads, wl.num_tokens, wl.head_dim), generator=gi, device=device,
                         dtype=torch.float32)
-        x.add_(field, alpha=0.5)
+        nv = wl.num_video_tokens
+        x[:, :, :nv].add_(field, alpha=0.5)
         if idx < 2:
-            _rope_(x, wl)
+            _rope_(x[:, :, :nv], wl)
         out.append(x.to(torch.bfloat16))
         del x
     return tuple(out)

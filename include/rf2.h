@@ -56,13 +56,21 @@ typedef enum {
  * short at the grid edge.  With first_frame_sink = 1 (section 3.4) frame 0 is
  * moved behind frames 1..F-1, every query block holding a first-frame token
  * keeps every key block, and every query block keeps every key block holding
- * a first-frame token. */
+ * a first-frame token.  Text tokens (text_tokens > 0; sequence length
+ * N = frames*height*width + text_tokens) join that full-attention region
+ * (section 3.4 groups the first frame with the text tokens of multimodal
+ * models): with the sink on, the region starts at frame 0; with it off, at
+ * the first text token. */
 typedef struct {
     int32_t batch, heads, head_dim;     /* head_dim in {64, 128} */
     int32_t frames, height, width;      /* latent grid; frames = 1 for images */
     int32_t win_t, win_h, win_w;        /* permutation window, each >= 1 */
     int32_t block;                      /* query/key block size; 64 */
     int32_t first_frame_sink;           /* 0 or 1 */
+    int32_t text_tokens;                /* >= 0: text tokens of a joint video-text attention, stored
+                                           after the frames*height*width video tokens; they stay
+                                           after the permuted video (behind frame 0) and take part
+                                           in full attention as sink rows and columns (section 3.4) */
 } rf2_geometry;
 
 /* Derived sizes (rf2_query). */

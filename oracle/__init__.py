@@ -91,22 +91,30 @@ def keep_count(keep: float, Tb: int) -> int:
     return max(1, min(Tb, n))
 
 
-def sink_start(T: int, H: int, W: int, sink: bool) -> int:
-    """First sink block, or -1 when the sink is off.
+def sink_start(T: int, H: int, W: int, sink: bool, text: int = 0) -> int:
+    """First sink block, or -1 when there is no full-attention region.
 
     With a single frame every token is a first-frame token, so every block is
-    a sink block (start 0) and the mask is full."""
-    if not sink:
-        return -1
-    return ((T - 1) * H * W) // BLOCK
+    a sink block (start 0) and the mask is full.  Text tokens of a joint
+    video-text attention sit after the video and join the full-attention
+    region (section 3.4 groups the first frame with them): with the sink off
+    the region starts at the first text token."""
+    if sink:
+        return ((T - 1) * H * W) // BLOCK
+    if text > 0:
+        return (T * H * W) // BLOCK
+    return -1
 
 
-def permutation(T: int, H: int, W: int, wt: int, wh: int, ww: int, sink: bool) -> np.ndarray:
-    """perm[p] = original [F,H,W] index of the token at permuted position p."""
-    perm = np.empty(T * H * W, dtype=np.int64)
+def permutation(T: int, H: int, W: int, wt: int, wh: int, ww: int, sink: bool, text: int = 0) -> np.ndarray:
+    """perm[p] = original index of the token at permuted position p: the
+    [F,H,W] video tokens in window order, then the `text` tokens unmoved."""
+    nv = T * H * W
+    perm = np.empty(nv + text, dtype=np.int64)
     rc = _load().orc_permutation(T, H, W, wt, wh, ww, int(bool(sink)), _ptr(perm))
     if rc != 0:
         raise ValueError(f"orc_permutation failed ({rc})")
+    perm[nv:] = np.arange(nv, nv + text)
     return perm
 
 
@@ -189,12 +197,12 @@ def select_cdf(S: np.ndarray, tau: float, sink_first: int):
     return mask, cum, bnd
 
 
-def predict_mask_cdf(qp, kp, tau: float, T: int, H: int, W: int, sink: bool):
+def predict_mask_cdf(qp, kp, tau: float, T: int, H: int, W: int, sink: bool, text: int = 0):
     """Mask prediction with CDF-threshold selection: means, scores, CDF + sink.
     Returns (mask, cum, bnd, S)."""
     qm, km = block_means(qp), block_means(kp)
     S = pooled_scores(qm, km)
-    mask, cum, bnd = select_cdf(S, tau, sink_start(T, H, W, sink))
+    mask, cum, bnd = select_cdf(S, tau, sink_start(T, H, W, sink, text))
     return mask, cum, bnd, S
 
 
@@ -232,11 +240,11 @@ def full_attention_output(qp, kp, vp, mask):
             lse.reshape(BH, Tb * BLOCK)[:, :N].copy())
 
 
-def predict_mask(qp, kp, keep: float, T: int, H: int, W: int, sink: bool):
+def predict_mask(qp, kp, keep: float, T: int, H: int, W: int, sink: bool, text: int = 0):
     """Steps of mask prediction in the paper's order: means, scores, top-n + sink.
     Returns (mask, thr, S)."""
     qm, km = block_means(qp), block_means(kp)
     S = pooled_scores(qm, km)
     Tb = S.shape[-1]
-    mask, thr = select_blocks(S, keep_count(keep, Tb), sink_start(T, H, W, sink))
+    mask, thr = select_blocks(S, keep_count(keep, Tb), sink_start(T, H, W, sink, text))
     return mask, thr, S

@@ -74,13 +74,13 @@ def check_csr(mask: rf2.BlockMask, sink_first: int):
         assert rs[r] == exp
 
 
-def compare_masks(gpu_dense: np.ndarray, qp_bits, kp_bits, keep, T, H, W, sink):
+def compare_masks(gpu_dense: np.ndarray, qp_bits, kp_bits, keep, T, H, W, sink, text=0):
     """Bit-exact mask parity outside the tie band.  Returns (excluded, compared)."""
-    omask, thr, S = oracle.predict_mask(qp_bits, kp_bits, keep, T, H, W, sink)
+    omask, thr, S = oracle.predict_mask(qp_bits, kp_bits, keep, T, H, W, sink, text)
     omask = omask.reshape(gpu_dense.shape)
     S = S.reshape(gpu_dense.shape)
     thr = thr.reshape(gpu_dense.shape[:2])
-    s0 = oracle.sink_start(T, H, W, sink)
+    s0 = oracle.sink_start(T, H, W, sink, text)
     Tb = gpu_dense.shape[-1]
     band = np.abs(S - thr[..., None]) <= TIE_BAND
     if s0 >= 0:

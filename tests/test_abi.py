@@ -50,7 +50,7 @@ def test_query_matches_oracle_readings(L, name):
     assert sz.num_tokens == N
     assert sz.num_blocks == oracle.num_blocks(N)
     assert sz.n_keep == oracle.keep_count(wl.keep, sz.num_blocks)
-    assert sz.sink_first == oracle.sink_start(wl.frames, wl.height, wl.width, wl.sink)
+    assert sz.sink_first == oracle.sink_start(wl.frames, wl.height, wl.width, wl.sink, wl.text_tokens)
     Tb = sz.num_blocks
     n_sink = 0 if sz.sink_first < 0 else Tb - sz.sink_first
     assert sz.row_capacity == min(Tb, sz.n_keep + n_sink)
@@ -80,6 +80,21 @@ def test_permutation_index_matches_oracle(L):
             (T, H, W, wt, wh, ww, sink)
 
 
+def test_permutation_index_with_text_matches_oracle(L):
+    rng = np.random.default_rng(3)
+    cases = [(21, 30, 52, 4, 4, 4, True, 256), (1, 64, 64, 1, 8, 8, False, 512), (4, 16, 16, 1, 8, 8, True, 77)]
+    for _ in range(60):
+        T, H, W, wt, wh, ww, sink = random_grid_case(rng)
+        cases.append((T, H, W, wt, wh, ww, sink, int(rng.integers(0, 200))))
+    for (T, H, W, wt, wh, ww, sink, text) in cases:
+        g = rf2.make_geometry(1, 1, 64, T, H, W, wt, wh, ww, sink, text=text)
+        assert np.array_equal(rf2.permutation_index(g), oracle.permutation(T, H, W, wt, wh, ww, sink, text)), \
+            (T, H, W, wt, wh, ww, sink, text)
+        sz = rf2.query(g, 0.3)
+        assert sz.num_tokens == T * H * W + text
+        assert sz.sink_first == oracle.sink_start(T, H, W, sink, text)
+
+
 def _status(fn, *args):
     return fn(*args)
 
@@ -93,6 +108,7 @@ def test_host_validation(L):
     bad_win = rf2.make_geometry(1, 2, 64, 4, 16, 16, 0, 8, 8, True)
     bad_sink = rf2.make_geometry(1, 2, 64, 4, 16, 16, 1, 8, 8, True)
     bad_sink.first_frame_sink = 2
+    bad_text = rf2.make_geometry(1, 2, 64, 4, 16, 16, 1, 8, 8, True, text=-1)
     huge = rf2.make_geometry(1, 1, 64, 100, 64, 64, 1, 8, 8, False)    # T_b > 4096
     sz = rf2.Sizes()
     assert L.rf2_query(G(good), 0.5, G(sz)) == rf2.RF2_OK
@@ -106,6 +122,7 @@ def test_host_validation(L):
     assert L.rf2_query(G(huge), 0.5, G(sz)) == rf2.RF2_ERR_UNSUPPORTED
     assert L.rf2_query(G(bad_win), 0.5, G(sz)) == rf2.RF2_ERR_INVALID_ARGUMENT
     assert L.rf2_query(G(bad_sink), 0.5, G(sz)) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_query(G(bad_text), 0.5, G(sz)) == rf2.RF2_ERR_INVALID_ARGUMENT
     # permute / unpermute
     for fn in (L.rf2_permute, L.rf2_unpermute):
         assert fn(G(good), None, fake, None) == rf2.RF2_ERR_INVALID_ARGUMENT

@@ -30,15 +30,15 @@ def _built():
     torch.cuda.synchronize()
 
 
-def compare_cdf_masks(gpu_dense, qp_b, kp_b, tau, T, H, W, sink):
+def compare_cdf_masks(gpu_dense, qp_b, kp_b, tau, T, H, W, sink, text=0):
     """Exact comparison outside the boundary band.  Returns (excluded, compared)."""
-    omask, cum, bnd, S = oracle.predict_mask_cdf(qp_b, kp_b, tau, T, H, W, sink)
+    omask, cum, bnd, S = oracle.predict_mask_cdf(qp_b, kp_b, tau, T, H, W, sink, text)
     Tb = gpu_dense.shape[-1]
     omask = omask.reshape(gpu_dense.shape)
     S = S.reshape(gpu_dense.shape)
     cum = cum.reshape(gpu_dense.shape[:2] + (2,))
     bnd = bnd.reshape(gpu_dense.shape[:2])
-    s0 = oracle.sink_start(T, H, W, sink)
+    s0 = oracle.sink_start(T, H, W, sink, text)
     excl = np.abs(S - bnd[..., None]) <= BAND
     near = (np.abs(cum[..., 0] - tau) <= BAND) | (np.abs(cum[..., 1] - tau) <= BAND)
     for bh, i in zip(*np.nonzero(near)):
@@ -85,6 +85,7 @@ def _cases():
         ("qwen_image", WORKLOADS["qwen_image"], 0.4),
         ("tau_one", W("c4", 1, 2, 64, 2, 12, 16, 2, 4, 4, 1.0, True, (24, 20, 20)), 1.0),
         ("tau_tiny", W("c5", 1, 2, 128, 3, 16, 16, 1, 8, 8, 0.01, True, (44, 42, 42)), 1e-4),
+        ("text_nosink", W("c6", 1, 2, 64, 2, 8, 8, 2, 4, 4, 0.4, False, (24, 20, 20), 70), 0.4),
     ]
 
 
@@ -95,7 +96,7 @@ def test_cdf_small_parity(name, wl, tau):
     check_csr(out["mask"], sz.sink_first)
     dense = out["mask"].dense()
     excluded, compared = compare_cdf_masks(dense, bits(out["qp"]), bits(out["kp"]), tau, wl.frames, wl.height,
-                                           wl.width, wl.sink)
+                                           wl.width, wl.sink, wl.text_tokens)
     # at most the two boundary blocks of each row, plus score ties
     assert excluded <= 2 * dense.shape[0] * dense.shape[1] + 0.01 * compared
     e = attention_errors(out["op"], bits(out["qp"]), bits(out["kp"]), bits(out["vp"]), dense)
@@ -108,7 +109,7 @@ def test_cdf_video480p_full_size():
     dense = out["mask"].dense()
     check_csr(out["mask"], out["mask"].sizes.sink_first)
     excluded, compared = compare_cdf_masks(dense, bits(out["qp"]), bits(out["kp"]), 0.2, wl.frames, wl.height,
-                                           wl.width, wl.sink)
+                                           wl.width, wl.sink, wl.text_tokens)
     print(f"video480p cdf: mask compared exactly on {compared} blocks, {excluded} in the boundary band")
     assert excluded <= 0.01 * compared
     rc = out["mask"].row_count.cpu().numpy()

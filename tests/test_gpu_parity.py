@@ -30,7 +30,7 @@ def _built():
 
 
 def _perm_of(wl):
-    return oracle.permutation(wl.frames, wl.height, wl.width, wl.win_t, wl.win_h, wl.win_w, wl.sink)
+    return oracle.permutation(wl.frames, wl.height, wl.width, wl.win_t, wl.win_h, wl.win_w, wl.sink, wl.text_tokens)
 
 
 def _small_cases():
@@ -47,6 +47,10 @@ def _small_cases():
         ("keep_one", W("r6", 1, 2, 128, 3, 16, 16, 1, 8, 8, 0.01, True, (44, 42, 42))),
         ("keep_all", W("r7", 1, 2, 64, 2, 12, 16, 2, 4, 4, 1.0, True, (24, 20, 20))),
         ("odd_blocks", W("r8", 1, 2, 128, 1, 24, 40, 1, 8, 8, 0.4, False, (0, 64, 64))),
+        # text tokens of a joint video-text attention (section 3.4)
+        ("text_sink", W("t1", 1, 2, 128, 3, 8, 8, 1, 8, 8, 0.3, True, (44, 42, 42), 77)),
+        ("text_nosink", W("t2", 1, 2, 64, 2, 8, 8, 2, 4, 4, 0.4, False, (24, 20, 20), 70)),
+        ("image_text", W("t3", 1, 2, 128, 1, 16, 16, 1, 8, 8, 0.3, False, (0, 64, 64), 100)),
     ]
 
 
@@ -64,7 +68,8 @@ def test_small_case_parity(name, wl):
     sz = out["mask"].sizes
     check_csr(out["mask"], sz.sink_first)
     dense = out["mask"].dense()
-    compare_masks(dense, bits(out["qp"]), bits(out["kp"]), wl.keep, wl.frames, wl.height, wl.width, wl.sink)
+    compare_masks(dense, bits(out["qp"]), bits(out["kp"]), wl.keep, wl.frames, wl.height, wl.width, wl.sink,
+                  wl.text_tokens)
     # attention under the GPU's mask, and the unpermuted output
     e = attention_errors(out["op"], bits(out["qp"]), bits(out["kp"]), bits(out["vp"]), dense, lse=out["lse"])
     assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, e
@@ -82,7 +87,8 @@ def test_image_parity(name):
     assert np.array_equal(bits(out["kp"]), oracle.permute(bits(k), perm))
     check_csr(out["mask"], -1)
     dense = out["mask"].dense()
-    compare_masks(dense, bits(out["qp"]), bits(out["kp"]), wl.keep, 1, wl.height, wl.width, False)
+    compare_masks(dense, bits(out["qp"]), bits(out["kp"]), wl.keep, 1, wl.height, wl.width, False,
+                  wl.text_tokens)
     Tb = wl.num_blocks
     items = [(bh, i) for bh in (0, 11, 23) for i in range(Tb)]
     e = attention_errors(out["op"], bits(out["qp"]), bits(out["kp"]), bits(out["vp"]), dense, items=items)
@@ -134,7 +140,7 @@ def test_constant_value_rows():
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged_d128", "ragged_d64_nosink", "one_block", "single_frame_sink",
-                                  "odd_blocks", "video720p"])
+                                  "odd_blocks", "text_nosink", "video720p"])
 def test_fused_permute_pool_matches_unfused(name):
     """rf2_permute_qk_pool writes the same Qp/Kp as rf2_permute and the same
     block means as the mask path's own pooling, bit for bit, so the predicted
@@ -195,7 +201,7 @@ def test_random_geometries():
         assert np.array_equal(bits(out["qp"]), oracle.permute(bits(q), _perm_of(wl))), wl
         dense = out["mask"].dense()
         check_csr(out["mask"], out["mask"].sizes.sink_first)
-        compare_masks(dense, bits(out["qp"]), bits(out["kp"]), wl.keep, T, H, W, wl.sink)
+        compare_masks(dense, bits(out["qp"]), bits(out["kp"]), wl.keep, T, H, W, wl.sink, wl.text_tokens)
         e = attention_errors(out["op"], bits(out["qp"]), bits(out["kp"]), bits(out["vp"]), dense)
         assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, (wl, e)
 
@@ -212,7 +218,8 @@ def _full_size(name, n_random_blocks, n_sink_blocks):
     del q, k, v
     sz = out["mask"].sizes
     dense = out["mask"].dense()
-    excluded, compared = compare_masks(dense, qp_b, kp_b, wl.keep, wl.frames, wl.height, wl.width, wl.sink)
+    excluded, compared = compare_masks(dense, qp_b, kp_b, wl.keep, wl.frames, wl.height, wl.width, wl.sink,
+                                       wl.text_tokens)
     # Blocks inside the tie band are excluded from the exact comparison; on
     # these inputs they are a fraction of a percent (pooled scores cluster).
     print(f"{name}: mask compared exactly on {compared} blocks, {excluded} in the 1e-5 tie band")
@@ -230,6 +237,10 @@ def _full_size(name, n_random_blocks, n_sink_blocks):
 
 def test_video480p_full_size():
     _full_size("video480p", 48, 4)
+
+
+def test_video480p_text_full_size():
+    _full_size("video480p_text", 32, 4)
 
 
 def test_video720p_full_size():

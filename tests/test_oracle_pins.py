@@ -14,6 +14,7 @@ import pytest
 import torch
 
 import oracle
+from image_dits_b200.workload import random_grid_case
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -323,3 +324,48 @@ def test_cdf_tau_one_keeps_everything_and_sink():
         kept = np.nonzero(mask[0, i, :20])[0]
         if kept.size:
             assert s[i, kept].min() >= np.sort(s[i, :20])[::-1][kept.size - 1]
+
+
+# ---- text tokens of a joint video-text attention (section 3.4) -------------------------------
+
+
+def test_text_geometry_golden():
+    with open(os.path.join(GOLDEN, "text_geometry.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    assert rows
+    for r in rows:
+        F, H, W, text, sink = int(r[0]), int(r[1]), int(r[2]), int(r[3]), bool(int(r[4]))
+        N, Tb, s0 = int(r[6]), int(r[7]), int(r[8])
+        assert F * H * W + text == N
+        assert oracle.num_blocks(N) == Tb
+        assert oracle.sink_start(F, H, W, sink, text) == s0
+
+
+def test_text_tokens_keep_their_place():
+    """Text tokens follow the permuted video unmoved; the video part is the
+    text-free permutation."""
+    rng = np.random.default_rng(9)
+    for _ in range(30):
+        T, H, W, wt, wh, ww, sink = random_grid_case(rng, 1500)
+        text = int(rng.integers(1, 100))
+        nv = T * H * W
+        perm = oracle.permutation(T, H, W, wt, wh, ww, sink, text)
+        assert np.array_equal(perm[:nv], oracle.permutation(T, H, W, wt, wh, ww, sink))
+        assert np.array_equal(perm[nv:], np.arange(nv, nv + text))
+
+
+def test_text_sink_rows_and_columns():
+    """With text tokens and the first-frame sink off, the blocks from the first
+    text token on are full rows and are kept by every row."""
+    rng = np.random.default_rng(10)
+    T, H, W, text = 2, 8, 8, 70                         # N = 198, T_b = 4, text from token 128 (block 2)
+    s0 = oracle.sink_start(T, H, W, False, text)
+    assert s0 == 2
+    S = rng.normal(size=(1, 4, 4))
+    mask, _ = oracle.select_blocks(S, 1, s0)
+    assert mask[0, 2:].all() and mask[0, :, 2:].all()
+    # top-1 runs over every key block: a non-sink row keeps its best block when that
+    # block is not already a sink column
+    for i in range(2):
+        best = int(np.argmax(S[0, i]))
+        assert mask[0, i, :2].sum() == (1 if best < 2 else 0)
