@@ -249,3 +249,30 @@ def test_video720p_full_size():
 
 def test_device_status_clean():
     assert rf2.device_status() == rf2.RF2_OK
+
+
+@pytest.mark.parametrize("name,chunks,tau", [("tiny", 2, None), ("image", 5, None), ("video480p_text", 4, None),
+                                             ("video480p", 3, 0.2)])
+def test_host_pipeline_matches_device_path(name, chunks, tau):
+    """HostPipeline (head chunks, copies overlapped with compute) gives the same
+    output bits as the single device call, over two back-to-back runs."""
+    wl = WORKLOADS[name]
+    q, k, v = make_qkv(wl, "cuda", seed=4)
+    g = rf2.geometry_of(wl)
+    if tau is None:
+        ref, _ = rf2.rainfusion_attention(g, q, k, v, wl.keep)
+    else:
+        mask, ws = rf2.alloc_mask(g, 1.0, q.device)
+        qp, kp = rf2.permute_qk_pool(g, q, k, ws)
+        rf2.predict_mask_cdf_pooled(g, tau, mask, ws)
+        ref = rf2.unpermute(g, rf2.block_sparse_attn(g, qp, kp, rf2.permute(g, v), mask))
+    torch.cuda.synchronize()
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty_like(hq).pin_memory()
+    pipe = rf2.HostPipeline(g, keep=None if tau is not None else wl.keep, tau=tau, chunks=chunks)
+    for _ in range(2):
+        ho.zero_()
+        pipe.run(hq, hk, hv, ho)
+        pipe.synchronize()
+        assert torch.equal(ho.view(torch.int16), ref.cpu().view(torch.int16))
+    assert rf2.device_status() == rf2.RF2_OK
