@@ -108,10 +108,32 @@ struct AttnArgs {
 
 // 32 scores of one row -> 16 packed bf16 pairs of P = 2^(s*sl2 - m), adding
 // the fp32 probabilities to sum4.  `nvalid` < 32 masks the tail columns.
+#ifndef RF2_EXP_PACKED
+#define RF2_EXP_PACKED 1
+#endif
+
 template <bool kMasked>
 __device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], float sl2, float neg_mu, int nvalid,
                                           uint32_t (&pk)[16], float (&sum4)[4])
 {
+    if (RF2_EXP_PACKED) {
+        // x = s*sl2 - m and the row sums two lanes at a time (fma/add.f32x2)
+        const float2 sc = make_float2(sl2, sl2), mu = make_float2(neg_mu, neg_mu);
+        float2 acc[2] = {make_float2(sum4[0], sum4[1]), make_float2(sum4[2], sum4[3])};
+        #pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc, mu);
+            float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (kMasked) {
+                p.x = (c < nvalid) ? p.x : 0.f;
+                p.y = (c + 1 < nvalid) ? p.y : 0.f;
+            }
+            acc[(c >> 1) & 1] = fadd2(acc[(c >> 1) & 1], p);
+            pk[c >> 1] = pack_bf16x2(p.x, p.y);
+        }
+        sum4[0] = acc[0].x; sum4[1] = acc[0].y; sum4[2] = acc[1].x; sum4[3] = acc[1].y;
+        return;
+    }
     #pragma unroll
     for (int c = 0; c < 32; c += 2) {
         const float x0 = fmaf(__uint_as_float(s[c]), sl2, neg_mu);
