@@ -16,6 +16,9 @@
 //                     (equal scores: lower j), union the sink columns, and
 //                     write the row as an ascending CSR list.  Sink rows keep
 //                     every column.
+// select_reg_kernel   the same selection with the row's keys in registers
+//                     (bisection with exact counts), used for rows of up to
+//                     512 key blocks.
 // select_cdf_kernel   the CDF-threshold alternative to top-n (see below).
 #pragma once
 #include "geometry.cuh"
@@ -500,6 +503,81 @@ __global__ void __launch_bounds__(kSelThreads) select_from_scores_kernel(const f
     uint32_t* hist = hist_all + warp * 256;
     for (int r = warp; r < nrows; r += kSelThreads / 32)
         select_row(keys + (size_t)r * Tb, hist, mg, bh, i0 + r, lane, row_start, row_count, col_idx, keep_all);
+}
+
+// Top-n selection with the row's keys in registers (rows of up to 32*KPL key
+// blocks): lane l holds the keys of j = l, l+32, ...  The threshold key, the
+// n-th largest, is found by bisection over the row's key range with exact
+// counts (each probe: KPL compares per lane and a warp sum), so a row costs
+// about (bits below the row's common prefix) probes of pure ALU work, no
+// shared memory and no atomics.  Equal keys go to the lowest j; output as in
+// select_row.  Same result as select_row.
+template <int KPL>
+__global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __restrict__ S, int32_t ld_s,
+                                                                 int32_t* __restrict__ row_start,
+                                                                 int32_t* __restrict__ row_count,
+                                                                 int32_t* __restrict__ col_idx, MaskGeo mg,
+                                                                 int64_t h0)
+{
+    const int Tb = mg.Tb;
+    const int lane = threadIdx.x & 31;
+    const int64_t hl = blockIdx.y;
+    const int64_t bh = h0 + hl;
+    const int i = blockIdx.x * (kSelThreads / 32) + (threadIdx.x >> 5);
+    if (i >= Tb) return;                                   // whole warp
+    const int64_t rs = row_offset(mg, bh, i);
+    const int64_t row_id = bh * Tb + i;
+    int32_t* out = col_idx + rs;
+    if (i >= mg.sink_first || mg.n_keep >= Tb) {
+        for (int j = lane; j < Tb; j += 32) out[j] = j;
+        if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = Tb; }
+        return;
+    }
+    const float* src = S + (hl * Tb + i) * (int64_t)ld_s;
+    uint32_t key[KPL];
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    #pragma unroll
+    for (int u = 0; u < KPL; ++u) {
+        const int j = u * 32 + lane;
+        key[u] = (j < Tb) ? float_order_key(src[j]) : 0u;  // 0: below every real key
+        if (j < Tb) { kmin = min(kmin, key[u]); kmax = max(kmax, key[u]); }
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const int n = mg.n_keep;
+    // largest K in [kmin, kmax] with #{key >= K} >= n (#{key >= kmin} = Tb >= n)
+    uint32_t lo = kmin, hi = kmax;
+    while (lo < hi) {
+        const uint32_t mid = lo + (uint32_t)(((uint64_t)hi - lo + 1) >> 1);
+        int c = 0;
+        #pragma unroll
+        for (int u = 0; u < KPL; ++u) c += (key[u] >= mid);
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (c >= n) lo = mid;
+        else hi = mid - 1;
+    }
+    const uint32_t thr = lo;
+    int gt = 0;
+    #pragma unroll
+    for (int u = 0; u < KPL; ++u) gt += (key[u] > thr);
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    int eq_left = n - gt;                                  // keys equal to thr that are kept
+    int written = 0;
+    #pragma unroll
+    for (int u = 0; u < KPL; ++u) {
+        const int j = u * 32 + lane;
+        if (u * 32 >= Tb) break;                           // uniform
+        const uint32_t k = key[u];
+        const bool eq = (j < Tb) && (k == thr);
+        const uint32_t eq_ballot = __ballot_sync(0xffffffffu, eq);
+        const int eq_rank = __popc(eq_ballot & ((1u << lane) - 1u));
+        const bool sel = (j < Tb) && (k > thr || (eq && eq_rank < eq_left) || j >= mg.sink_first);
+        eq_left -= __popc(eq_ballot);
+        const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[written + __popc(sel_ballot & ((1u << lane) - 1u))] = j;
+        written += __popc(sel_ballot);
+    }
+    if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = written; }
 }
 
 // CDF-threshold selection ("RainFusion2.0" section 2, online adaptive
