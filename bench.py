@@ -249,7 +249,7 @@ def run_reference(args, wl, rank):
     times, flops = [], 0.0
     desc = ""
     for s in range(args.steps):
-        f, dt, desc = oracle_sample(wl, seed=s, n_query_blocks=4)
+        f, dt, desc = oracle_sample(wl, seed=s, n_query_blocks=32)
         times.append(dt)
         flops += f
     total = sum(times)
