@@ -192,7 +192,9 @@ def oracle_sample(wl, seed=0, n_query_blocks=32, budget_s=None):
     K, V, the full mask of that head, and attention for a sample of query
     blocks (one of them a sink block).  With budget_s, attention runs in
     chunks of n_query_blocks random query blocks until that many seconds have
-    passed.  Returns (kept_flops, seconds, desc)."""
+    passed.  Returns (kept_flops, seconds, desc, stages): stages holds the
+    wall time of each step for the head (attention for the sampled blocks,
+    and extrapolated to all of the head's kept pairs)."""
     import oracle
     from image_dits_b200.workload import Workload
     one = Workload(wl.name, 1, 1, wl.head_dim, wl.frames, wl.height, wl.width, wl.win_t, wl.win_h, wl.win_w,
@@ -205,7 +207,9 @@ def oracle_sample(wl, seed=0, n_query_blocks=32, budget_s=None):
     t0 = time.perf_counter()
     perm = oracle.permutation(wl.frames, wl.height, wl.width, wl.win_t, wl.win_h, wl.win_w, wl.sink, wl.text_tokens)
     qp, kp, vp = oracle.permute(qb, perm), oracle.permute(kb, perm), oracle.permute(vb, perm)
+    t1 = time.perf_counter()
     mask, _, _ = oracle.predict_mask(qp, kp, wl.keep, wl.frames, wl.height, wl.width, wl.sink, wl.text_tokens)
+    t2 = time.perf_counter()
     Tb = wl.num_blocks
     rng = np.random.default_rng(seed)
     s0 = oracle.sink_start(wl.frames, wl.height, wl.width, wl.sink, wl.text_tokens)
@@ -224,18 +228,24 @@ def oracle_sample(wl, seed=0, n_query_blocks=32, budget_s=None):
             break
         chunk = order[pos:pos + n_query_blocks]
         pos += n_query_blocks
+    t3 = time.perf_counter()
     oracle.unpermute(qp, perm)
-    dt = time.perf_counter() - t0
+    t4 = time.perf_counter()
+    dt = t4 - t0
     last = N - 64 * (Tb - 1)
-    flops = 0.0
-    for i in blocks:
+
+    def block_flops(i):
         r = 64 if i < Tb - 1 else last
         m = mask.reshape(Tb, Tb)[i]
         c = 64 * int(m.sum()) - (64 - last) * int(m[Tb - 1])
-        flops += 4.0 * wl.head_dim * r * c
+        return 4.0 * wl.head_dim * r * c
+    flops = sum(block_flops(i) for i in blocks)
+    head_flops = sum(block_flops(i) for i in range(Tb))
+    stages = {"permute_qkv_s": t1 - t0, "predict_mask_s": t2 - t1, "attention_sample_s": t3 - t2,
+              "attention_head_s_extrapolated": (t3 - t2) * head_flops / flops, "unpermute_s": t4 - t3}
     desc = (f"1 of {wl.heads} heads: permutation of Q/K/V, the head's full block mask, attention for "
             f"{len(blocks)} of {Tb} query blocks (1 sink block), unpermute")
-    return flops, dt, desc
+    return flops, dt, desc, stages
 
 
 def run_reference(args, wl, rank):
@@ -249,7 +259,7 @@ def run_reference(args, wl, rank):
     times, flops = [], 0.0
     desc = ""
     for s in range(args.steps):
-        f, dt, desc = oracle_sample(wl, seed=s, n_query_blocks=32)
+        f, dt, desc, _ = oracle_sample(wl, seed=s, n_query_blocks=32)
         times.append(dt)
         flops += f
     total = sum(times)
@@ -540,9 +550,17 @@ def main():
         try:
             import oracle
             oracle.build()
-            f, dt, desc = oracle_sample(wl, budget_s=12.0)
+            f, dt, desc, st = oracle_sample(wl, budget_s=12.0)
+            heads = wl.batch * wl.heads
+            full = heads * (st["permute_qkv_s"] + st["predict_mask_s"] + st["attention_head_s_extrapolated"]
+                            + st["unpermute_s"])
             line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
-                                    "kind": "oracle", "cpu": cpu_info(), "seconds": dt, "sample": desc}
+                                    "kind": "oracle", "cpu": cpu_info(), "seconds": dt, "sample": desc,
+                                    "stages_per_head_s": st,
+                                    "full_call_s_extrapolated": full,
+                                    "note": "full_call_s_extrapolated = heads x (permute + mask + attention over "
+                                            "all of the head's kept pairs, extrapolated from the sample by kept "
+                                            "FLOPs + unpermute)"}
         except Exception as exc:  # the baseline must not hide the GPU line
             line["cpu_baseline"] = {"value": None, "error": repr(exc)}
 
