@@ -16,9 +16,9 @@
 //                     (equal scores: lower j), union the sink columns, and
 //                     write the row as an ascending CSR list.  Sink rows keep
 //                     every column.
-// select_reg_kernel   the same selection with the row's keys in registers
-//                     (bisection with exact counts), used for rows of up to
-//                     512 key blocks.
+// select_probe_kernel the same selection with the row's keys in registers
+//                     (a few counting probes, then an exact rank of the last
+//                     <= 32 candidates), used for rows of up to 512 key blocks.
 // select_cdf_kernel   the CDF-threshold alternative to top-n (see below).
 #pragma once
 #include "geometry.cuh"
@@ -505,22 +505,32 @@ __global__ void __launch_bounds__(kSelThreads) select_from_scores_kernel(const f
         select_row(keys + (size_t)r * Tb, hist, mg, bh, i0 + r, lane, row_start, row_count, col_idx, keep_all);
 }
 
-// Top-n selection with the row's keys in registers (rows of up to 32*KPL key
-// blocks): lane l holds the keys of j = l, l+32, ...  The threshold key, the
-// n-th largest, is found by bisection over the row's key range with exact
-// counts (each probe: KPL compares per lane and a warp sum), so a row costs
-// about (bits below the row's common prefix) probes of pure ALU work, no
-// shared memory and no atomics.  Equal keys go to the lowest j; output as in
-// select_row.  Same result as select_row.
-template <int KPL>
-__global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __restrict__ S, int32_t ld_s,
-                                                                 int32_t* __restrict__ row_start,
-                                                                 int32_t* __restrict__ row_count,
-                                                                 int32_t* __restrict__ col_idx, MaskGeo mg,
-                                                                 int64_t h0)
+// Inverse of float_order_key.
+__device__ __forceinline__ float order_key_float(uint32_t k)
 {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Top-n selection, keys in registers, few counting probes: the threshold key
+// (the n-th largest) is bracketed by keys lo < hi with #{key >= lo} >= n >
+// #{key >= hi}; each probe counts the keys at or above one candidate key
+// (KPL compares per lane and a warp sum).  Probes alternate between a guess
+// interpolated in score value from the bracket's counts (scores are smooth,
+// so a few probes narrow the bracket to a handful of keys) and a plain key
+// bisection (which bounds the probe count).  Once at most 32 keys lie in the
+// bracket they are gathered and ranked exactly with one warp-wide bitonic
+// sort.  Equal keys go to the lowest j; output as in select_row.
+template <int KPL>
+__global__ void __launch_bounds__(kSelThreads) select_probe_kernel(const float* __restrict__ S, int32_t ld_s,
+                                                                   int32_t* __restrict__ row_start,
+                                                                   int32_t* __restrict__ row_count,
+                                                                   int32_t* __restrict__ col_idx, MaskGeo mg,
+                                                                   int64_t h0)
+{
+    __shared__ uint32_t cand_all[kSelThreads];
     const int Tb = mg.Tb;
     const int lane = threadIdx.x & 31;
+    uint32_t* cand = cand_all + (threadIdx.x & ~31);
     const int64_t hl = blockIdx.y;
     const int64_t bh = h0 + hl;
     const int i = blockIdx.x * (kSelThreads / 32) + (threadIdx.x >> 5);
@@ -539,27 +549,71 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __
     #pragma unroll
     for (int u = 0; u < KPL; ++u) {
         const int j = u * 32 + lane;
-        key[u] = (j < Tb) ? float_order_key(src[j]) : 0u;  // 0: below every real key
+        key[u] = (j < Tb) ? float_order_key(src[j]) : 0u;
         if (j < Tb) { kmin = min(kmin, key[u]); kmax = max(kmax, key[u]); }
     }
     kmin = __reduce_min_sync(0xffffffffu, kmin);
     kmax = __reduce_max_sync(0xffffffffu, kmax);
     const int n = mg.n_keep;
-    // largest K in [kmin, kmax] with #{key >= K} >= n (#{key >= kmin} = Tb >= n)
-    uint32_t lo = kmin, hi = kmax;
-    while (lo < hi) {
-        const uint32_t mid = lo + (uint32_t)(((uint64_t)hi - lo + 1) >> 1);
+    auto count_ge = [&](uint32_t K) -> int {
         int c = 0;
         #pragma unroll
-        for (int u = 0; u < KPL; ++u) c += (key[u] >= mid);
-        c = __reduce_add_sync(0xffffffffu, c);
-        if (c >= n) lo = mid;
-        else hi = mid - 1;
+        for (int u = 0; u < KPL; ++u) c += (u * 32 + lane < Tb) && (key[u] >= K);
+        return __reduce_add_sync(0xffffffffu, c);
+    };
+    // bracket: [lo, hi) with count_ge(lo) = c_lo >= n > c_hi = count_ge(hi)
+    uint64_t lo = kmin, hi = (uint64_t)kmax + 1;
+    int c_lo = Tb, c_hi = 0;
+    #pragma unroll 1
+    for (int it = 0; it < 80 && c_lo - c_hi > 32 && hi - lo > 1; ++it) {
+        uint64_t mid;
+        if ((it & 1) == 0) {
+            const float vlo = order_key_float((uint32_t)lo), vhi = order_key_float((uint32_t)(hi - 1));
+            // the bracket's keys below the n-th largest, as a fraction of the
+            // bracket: place the guess that far up the bracket's value range
+            const float f = ((float)(c_lo - n) + 0.5f) / (float)(c_lo - c_hi);
+            mid = float_order_key(vlo + f * (vhi - vlo));
+        } else {
+            mid = lo + ((hi - lo) >> 1);
+        }
+        if (mid <= lo) mid = lo + 1;
+        if (mid >= hi) mid = hi - 1;
+        const int c = count_ge((uint32_t)mid);
+        if (c >= n) { lo = mid; c_lo = c; }
+        else { hi = mid; c_hi = c; }
     }
-    const uint32_t thr = lo;
+    uint32_t thr;
+    if (hi - lo <= 1) {
+        thr = (uint32_t)lo;
+    } else {
+        // at most 32 keys in [lo, hi): gather them and rank them exactly
+        int base = 0;
+        #pragma unroll
+        for (int u = 0; u < KPL; ++u) {
+            const bool in = (u * 32 + lane < Tb) && key[u] >= (uint32_t)lo && (uint64_t)key[u] < hi;
+            const uint32_t b = __ballot_sync(0xffffffffu, in);
+            if (in) cand[base + __popc(b & ((1u << lane) - 1u))] = key[u];
+            base += __popc(b);
+        }
+        __syncwarp();
+        uint32_t v = (lane < base) ? cand[lane] : 0u;       // 0 sorts below every candidate
+        // bitonic sort, descending over the 32 lanes
+        #pragma unroll
+        for (int k = 2; k <= 32; k <<= 1) {
+            #pragma unroll
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                const uint32_t o = __shfl_xor_sync(0xffffffffu, v, jj);
+                const bool desc = ((lane & k) == 0);
+                const bool lower = ((lane & jj) == 0);
+                v = (lower == desc) ? max(v, o) : min(v, o);
+            }
+        }
+        thr = __shfl_sync(0xffffffffu, v, n - c_hi - 1);      // rank n - c_hi within the bracket
+        __syncwarp();
+    }
     int gt = 0;
     #pragma unroll
-    for (int u = 0; u < KPL; ++u) gt += (key[u] > thr);
+    for (int u = 0; u < KPL; ++u) gt += (u * 32 + lane < Tb) && (key[u] > thr);
     gt = __reduce_add_sync(0xffffffffu, gt);
     int eq_left = n - gt;                                  // keys equal to thr that are kept
     int written = 0;

@@ -304,14 +304,13 @@ static int launch_select(const Checked& c, const MaskGeo& mg, const float* S, in
     return launch_status();
 }
 
-// Top-n selection with the row's keys in registers: KPL keys per lane.
 template <int KPL>
-static int launch_select_reg(const Checked& c, const MaskGeo& mg, const float* S, int64_t h0, int64_t g,
-                             int32_t* row_start, int32_t* row_count, int32_t* col_idx, cudaStream_t s)
+static int launch_select_probe(const Checked& c, const MaskGeo& mg, const float* S, int64_t h0, int64_t g,
+                               int32_t* row_start, int32_t* row_count, int32_t* col_idx, cudaStream_t s)
 {
     constexpr int rows_per_cta = kSelThreads / 32;
     dim3 grid((c.Tb + rows_per_cta - 1) / rows_per_cta, (unsigned)g);
-    select_reg_kernel<KPL><<<grid, kSelThreads, 0, s>>>(S, score_ld(c.Tb), row_start, row_count, col_idx, mg, h0);
+    select_probe_kernel<KPL><<<grid, kSelThreads, 0, s>>>(S, score_ld(c.Tb), row_start, row_count, col_idx, mg, h0);
     return launch_status();
 }
 
@@ -321,8 +320,12 @@ static int launch_select_topn(const Checked& c, const MaskGeo& mg, const float* 
     // Keys in registers pay off while a lane holds few of them (measured:
     // 11% faster at T_b = 512; at T_b = 1182, 40 keys per lane, the register
     // footprint halves occupancy and the shared-memory radix select is faster).
+    // Keys in registers pay off while a lane holds few of them (measured: the
+    // image shape's mask 19% faster, 480p equal; at T_b = 1182, 40 keys per
+    // lane, the register footprint halves occupancy and the shared-memory
+    // radix select is faster).
     if (RF2_SELECT_REG && c.Tb <= 32 * 16)
-        return launch_select_reg<16>(c, mg, S, h0, g, row_start, row_count, col_idx, s);
+        return launch_select_probe<16>(c, mg, S, h0, g, row_start, row_count, col_idx, s);
     return launch_select<8>(c, mg, S, h0, g, row_start, row_count, col_idx, s);
 }
 
