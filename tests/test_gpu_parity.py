@@ -8,6 +8,8 @@ Sizes span several tiles with ragged tails; the video workloads at full size
 are compared in full for the permutation and the mask, and on sampled query
 blocks for the attention output.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -137,6 +139,36 @@ def test_constant_value_rows():
     out = run_path(rf2.geometry_of(wl), q, k, v, wl.keep)
     err = (out["o"].float() - v.float()).abs().max().item()
     assert err <= 2 ** -7 * v.float().abs().max().item() + 1e-6
+
+
+@pytest.mark.parametrize("d,keep", [(128, 1.0), (128, 0.5), (64, 0.4)])
+def test_running_max_rescale(d, keep):
+    """Key blocks in four groups whose scores step up by about 9 (log2 units)
+    from one group to the next, and query rows alternating in sign: rows whose
+    scores rise raise their running max, and O is rescaled, at the group
+    boundaries, while the other rows of the same warp keep their first max;
+    under a sparse mask (chosen on the unmodified scores) the steps fall at
+    different entries for the two query blocks of a tile."""
+    rope = (44, 42, 42) if d == 128 else (24, 20, 20)
+    wl = Workload("rescale", 1, 2, d, 4, 16, 16, 2, 4, 4, keep, False, rope)
+    g = rf2.geometry_of(wl)
+    q, k, v = make_qkv(wl, "cuda", seed=11)
+    qp, kp, vp = rf2.permute(g, q), rf2.permute(g, k), rf2.permute(g, v)
+    mask = rf2.predict_mask(g, qp, kp, keep)
+    N, Tb = wl.num_tokens, wl.num_blocks
+    sl2 = math.log2(math.e) / math.sqrt(d)
+    A = 16.0
+    sign = torch.where(torch.arange(N, device="cuda") % 2 == 0, 1.0, -1.0)
+    qp[..., 0] = (A * sign).to(qp.dtype)
+    group = (torch.arange(N, device="cuda") // 64) * 4 // Tb
+    kp[..., 0] = (9.0 * group / (sl2 * A)).to(kp.dtype)
+    lse = torch.full((wl.heads * N,), float("nan"), device="cuda")
+    op = rf2.block_sparse_attn(g, qp, kp, vp, mask, lse=lse)
+    torch.cuda.synchronize()
+    assert rf2.device_status() == rf2.RF2_OK
+    e = attention_errors(op, bits(qp), bits(kp), bits(vp), mask.dense(), lse=lse)
+    assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, e
+    assert e["lse_max_abs"] <= 1e-3, e
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged_d128", "ragged_d64_nosink", "one_block", "single_frame_sink",
