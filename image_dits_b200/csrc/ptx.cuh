@@ -304,24 +304,6 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
-// 2^x on the FMA pipe, for softmax arguments (x <= 8): x = j + f with j the
-// nearest integer (adding 1.5*2^23 rounds x into the low mantissa bits) and
-// f in [-0.5, 0.5]; 2^f from a cubic fitted for least maximum relative error
-// on that interval (max rel. error 7.5e-5, well below bf16's 2^-9 half-ulp);
-// 2^j by adding j to the exponent field.  Arguments below -125 are clamped
-// (the result is then ~2^-125, nothing at bf16 / fp32-sum precision).
-__device__ __forceinline__ float exp2_poly(float x)
-{
-    x = fmaxf(x, -125.f);
-    const float kRound = 12582912.f;
-    const float t = x + kRound;
-    const float f = x - (t - kRound);
-    float p = fmaf(0.0551716685295105f, f, 0.2426111400127411f);
-    p = fmaf(p, f, 0.6932609677314758f);
-    p = fmaf(p, f, 0.9999280571937561f);
-    return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - __float_as_int(kRound)) << 23));
-}
-
 // Packed fp32 pairs (sm_100 fma.rn.f32x2 / add.rn.f32x2: two lanes of fp32
 // arithmetic per instruction).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
