@@ -98,7 +98,7 @@ struct AttnArgs {
     int32_t N;
     int32_t Tb;
     int32_t pairs;          // ceil(Tb / 2)
-    int32_t sink_pairs;     // pairs holding a sink block: scheduled first in each head
+    int32_t sink_pairs;     // pairs holding a sink block (the last ones of a head): scheduled early
     float scale_log2;       // log2(e) / sqrt(D)
 };
 
@@ -156,10 +156,31 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int lane = tid & 31;
     const int Tb = args.Tb;
 
-    // ---- work item: (bh, pair); sink pairs of a head first (they are the longest)
-    const int64_t bh = blockIdx.x / args.pairs;
-    const int u = (int)(blockIdx.x - bh * args.pairs);
-    const int pair = (u < args.sink_pairs) ? (args.pairs - 1 - u) : (u - args.sink_pairs);
+    // ---- work item (bh, pair).  The sink pairs of a head (full rows: the
+    // longest items) are launched just before the other pairs of the previous
+    // head, so they start early and the grid ends on short items, while the
+    // CTAs in flight use the K/V of at most two heads (L2-resident).
+    int64_t bh;
+    int pair;
+    {
+        const int P = args.pairs, S = args.sink_pairs;
+        const int64_t BH = gridDim.x / P;
+        const int64_t x = blockIdx.x;
+        if (x < S) {
+            bh = 0;
+            pair = P - 1 - (int)x;
+        } else {
+            const int64_t g = 1 + (x - S) / P;     // group g: sink pairs of head g, then the rest of head g - 1
+            const int r = (int)(x - S - (g - 1) * P);
+            if (g < BH && r < S) {
+                bh = g;
+                pair = P - 1 - r;
+            } else {
+                bh = g - 1;
+                pair = (g < BH) ? r - S : r;
+            }
+        }
+    }
     const int qb0 = 2 * pair;
     const bool has_b = (qb0 + 1) < Tb;
 
