@@ -156,28 +156,30 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int lane = tid & 31;
     const int Tb = args.Tb;
 
-    // ---- work item (bh, pair).  The sink pairs of a head (full rows: the
-    // longest items) are launched just before the other pairs of the previous
-    // head, so they start early and the grid ends on short items, while the
-    // CTAs in flight use the K/V of at most two heads (L2-resident).
+    // ---- work item (bh, pair).  A head's sink pairs (full rows: the longest
+    // items) are launched before its other pairs, so the CTAs in flight use
+    // the K/V of about one head (L2-resident); for the last two heads both
+    // heads' sink pairs come first, so the grid does not end on full rows.
     int64_t bh;
     int pair;
     {
         const int P = args.pairs, S = args.sink_pairs;
         const int64_t BH = gridDim.x / P;
         const int64_t x = blockIdx.x;
-        if (x < S) {
-            bh = 0;
-            pair = P - 1 - (int)x;
+        const int64_t tail0 = (BH >= 2) ? (BH - 2) * P : 0;   // first block of the last two heads
+        if (x < tail0 || BH < 2) {
+            bh = x / P;
+            const int u = (int)(x - bh * P);
+            pair = (u < S) ? (P - 1 - u) : (u - S);
         } else {
-            const int64_t g = 1 + (x - S) / P;     // group g: sink pairs of head g, then the rest of head g - 1
-            const int r = (int)(x - S - (g - 1) * P);
-            if (g < BH && r < S) {
-                bh = g;
-                pair = P - 1 - r;
+            const int t = (int)(x - tail0);                    // 0 .. 2P - 1
+            if (t < 2 * S) {
+                bh = BH - 2 + t / S;
+                pair = P - 1 - t % S;
             } else {
-                bh = g - 1;
-                pair = (g < BH) ? r - S : r;
+                const int v = t - 2 * S;                       // normal pairs of the two heads
+                bh = BH - 2 + v / (P - S);
+                pair = v % (P - S);
             }
         }
     }
