@@ -74,11 +74,11 @@ def kept_flops_from_mask(mask, wl) -> float:
 
 
 # DRAM bytes (read + write) per (token, head) of one block_sparse_attn_kernel<128>
-# launch, from an ncu capture at 480p (390.6 MB / (32,760 tokens x 12 heads)).  The
+# launch, from an ncu capture at 480p (391.2 MB / (32,760 tokens x 12 heads)).  The
 # kernel's DRAM traffic is its compulsory Q/K/V reads and O writes (K/V re-reads hit
 # L2), so it scales with the token-heads of the workload.  Re-measure whenever the
 # kernel changes.
-ATTN_DRAM_BYTES_PER_TOKEN_HEAD = (306.836e6 + 83.714e6) / (32760 * 12)
+ATTN_DRAM_BYTES_PER_TOKEN_HEAD = (306.926e6 + 84.263e6) / (32760 * 12)
 
 
 def mask_bytes(wl, mask) -> float:
