@@ -82,12 +82,18 @@ static int keep_count(double keep, int32_t Tb, int32_t* n)
 // fp32 arrays [2][BH][T_b][d], then the pooled-score buffer of one group of
 // heads [G][T_b][ld] (ld = T_b rounded up to 4 floats); heads are scored and
 // selected group by group so that the score buffer stays in L2 between the
-// two kernels.
-constexpr int64_t kScoreGroupHeads = 16;
+// two kernels: the workspace holds as many heads' scores as fit in
+// kScoreGroupBytes (at least one head).
+constexpr size_t kScoreGroupBytes = (size_t)96 << 20;
 static int32_t score_ld(int32_t Tb) { return (Tb + 3) & ~3; }
 static size_t mask_means_bytes(const Checked& c) { return ((size_t)2 * c.BH * c.Tb * c.D * sizeof(float) + 255) & ~(size_t)255; }
 static size_t score_head_bytes(const Checked& c) { return (size_t)c.Tb * score_ld(c.Tb) * sizeof(float); }
-static int64_t score_group_heads(int64_t BH) { return BH < kScoreGroupHeads ? BH : kScoreGroupHeads; }
+static int64_t score_group_heads(const Checked& c)
+{
+    int64_t g = (int64_t)(kScoreGroupBytes / score_head_bytes(c));
+    if (g < 1) g = 1;
+    return c.BH < g ? c.BH : g;
+}
 
 static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg, rf2_sizes* out)
 {
@@ -107,7 +113,7 @@ static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg
         out->row_capacity = mg.cap;
         out->num_rows = c.BH * c.Tb;
         out->col_idx_capacity = total;
-        out->mask_workspace_bytes = 2 * mask_means_bytes(c) + (size_t)score_group_heads(c.BH) * score_head_bytes(c);
+        out->mask_workspace_bytes = 2 * mask_means_bytes(c) + (size_t)score_group_heads(c) * score_head_bytes(c);
     }
     return RF2_OK;
 }
@@ -346,7 +352,8 @@ static int launch_select_cdf(const Checked& c, const MaskGeo& mg, const float* S
 
 // Block means, then per group of heads the tensor-core scores and the
 // selection.  `ws` holds the means followed by a score buffer for as many
-// heads (at most kScoreGroupHeads) as `ws_bytes` allows.
+// heads as `ws_bytes` allows, at most kScoreGroupBytes of scores and at most
+// as many heads as give the score kernel one item per SM.
 // Workspace pointers of the mask path; G = heads scored per group.
 struct MaskWs {
     float* means_hi;
@@ -360,7 +367,13 @@ static int mask_ws(const Checked& c, void* ws, size_t ws_bytes, MaskWs* w)
     const size_t mb = mask_means_bytes(c);
     if (ws_bytes < 2 * mb + score_head_bytes(c)) return RF2_ERR_INSUFFICIENT_WORKSPACE;
     int64_t G = (int64_t)((ws_bytes - 2 * mb) / score_head_bytes(c));
-    if (G > score_group_heads(c.BH)) G = score_group_heads(c.BH);
+    if (G > score_group_heads(c)) G = score_group_heads(c);
+    // one round of the persistent score kernel: a group's (head, 128-row tile)
+    // items at most one per SM (160 items on 148 SMs would take two rounds)
+    const int64_t tiles = (c.Tb + 127) / 128;
+    int64_t round_heads = num_sms() / tiles;
+    if (round_heads < 1) round_heads = 1;
+    if (G > round_heads) G = round_heads;
     w->means_hi = reinterpret_cast<float*>(ws);
     w->means_lo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + mb);
     w->S = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 2 * mb);

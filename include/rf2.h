@@ -84,7 +84,8 @@ typedef struct {
     int64_t col_idx_capacity;    /* length of col_idx */
     size_t  mask_workspace_bytes;/* scratch for rf2_predict_mask: the block means as a
                                     tf32 hi/lo pair of fp32 arrays, then the pooled
-                                    scores of up to 16 heads at a time */
+                                    scores of as many heads as fit in 96 MiB (at least
+                                    one head; all of them when they fit) */
 } rf2_sizes;
 
 /* Human-readable name of a status code (static string, never NULL). */
