@@ -643,6 +643,55 @@ int rf2_predict_mask_cdf_pooled(const rf2_geometry* geom, double tau, int32_t* r
                                (float)tau);
 }
 
+// Self-test of the timeout path: one CTA of two warps, each waiting (lane 0)
+// on its own mbarrier that nothing ever completes.  Warp 0 gives up after
+// `limit_ns`, records the timeout in the status word and raises the CTA's
+// abort flag; warp 1 (no time limit of its own beyond the usual one) must
+// leave through that flag.  Nothing faults; both waits end.
+static __global__ void selftest_timeout_kernel(uint64_t limit_ns, int* status, int* left)
+{
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bars[0]), 1);
+        mbar_init(smem_u32(&bars[1]), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (lane == 0) {
+        const bool ok = mbar_wait(smem_u32(&bars[warp]), 0, &abort_flag, status,
+                                  warp == 0 ? limit_ns : kWaitLimitNs);
+        if (!ok) atomicAdd(left, 1);
+    }
+}
+
+__device__ int g_selftest_given_up;
+
+static int* selftest_counter()
+{
+    int* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_selftest_given_up) != cudaSuccess) return nullptr;
+    return p;
+}
+
+int rf2_selftest_wait_timeout(uint32_t limit_us, int32_t* waits_given_up, void* stream)
+{
+    if (!waits_given_up || limit_us == 0 || limit_us > 1000000) return RF2_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int* status = status_word_ptr();
+    int* left = selftest_counter();
+    if (!status || !left) return RF2_ERR_CUDA;
+    if (cudaMemsetAsync(left, 0, sizeof(int), s) != cudaSuccess) return RF2_ERR_CUDA;
+    selftest_timeout_kernel<<<1, 64, 0, s>>>((uint64_t)limit_us * 1000u, status, left);
+    const int r = launch_status();
+    if (r != RF2_OK) return r;
+    if (cudaMemcpyAsync(waits_given_up, left, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return RF2_ERR_CUDA;
+    return cudaStreamSynchronize(s) == cudaSuccess ? RF2_OK : RF2_ERR_CUDA;
+}
+
 int rf2_device_status(void* stream)
 {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -28,7 +28,7 @@ EXPORTED = (
     "rf2_status_string", "rf2_query", "rf2_permutation_index", "rf2_permute", "rf2_unpermute",
     "rf2_predict_mask", "rf2_predict_mask_static", "rf2_permute_qk_pool", "rf2_predict_mask_pooled",
     "rf2_predict_mask_cdf", "rf2_predict_mask_cdf_pooled",
-    "rf2_block_sparse_attn", "rf2_device_status",
+    "rf2_block_sparse_attn", "rf2_device_status", "rf2_selftest_wait_timeout",
 )
 
 
@@ -83,6 +83,7 @@ def lib():
         L.rf2_predict_mask_cdf_pooled.argtypes = [G, f64, vp, vp, vp, vp, sz, vp]
         L.rf2_block_sparse_attn.argtypes = [G, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.rf2_device_status.argtypes = [vp]
+        L.rf2_selftest_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.POINTER(ctypes.c_int32), vp]
         for name in EXPORTED:
             if name != "rf2_status_string":
                 getattr(L, name).restype = i32
@@ -274,6 +275,17 @@ def block_sparse_attn(geom: Geometry, qp, kp, vp, mask: BlockMask, out: torch.Te
 def device_status(stream=None) -> int:
     """Synchronize and return (and clear) the device status word."""
     return int(lib().rf2_device_status(_stream(stream)))
+
+
+def selftest_wait_timeout(limit_us: int = 1000, stream=None) -> int:
+    """Run the library's timeout self-test (a bounded wait on a barrier that
+    nothing completes, and a second wait left through the abort flag); returns
+    how many of the two waits gave up.  The timeout is then in the device
+    status word (``device_status()`` returns RF2_ERR_TIMEOUT once)."""
+    n = ctypes.c_int32(-1)
+    _check(lib().rf2_selftest_wait_timeout(ctypes.c_uint32(int(limit_us)), ctypes.byref(n), _stream(stream)),
+           "rf2_selftest_wait_timeout")
+    return int(n.value)
 
 
 def rainfusion_attention(geom: Geometry, q, k, v, keep: float, stream=None):

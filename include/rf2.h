@@ -208,6 +208,18 @@ int rf2_block_sparse_attn(const rf2_geometry* geom, const void* qp_bf16, const v
  * kernel's bounded wait ran out since the last call. */
 int rf2_device_status(void* stream);
 
+/* Self-test of failure detection (tests only).  Launches, on `stream`, one
+ * CTA of two warps that wait on mbarriers nothing completes: the first gives
+ * up after `limit_us` microseconds (1 .. 1,000,000), records RF2_ERR_TIMEOUT in
+ * the device status word (read it with rf2_device_status) and raises the
+ * CTA's abort flag, through which the second leaves too -- the same bounded
+ * waits and abort path every kernel of the library uses.  Nothing faults and
+ * the context stays usable.  Synchronizes `stream`; *waits_given_up (host)
+ * receives the number of waits that ended without their barrier (2 when the
+ * path works).  Returns RF2_ERR_INVALID_ARGUMENT for a null pointer or a limit
+ * out of range. */
+int rf2_selftest_wait_timeout(uint32_t limit_us, int32_t* waits_given_up, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

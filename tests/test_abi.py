@@ -184,3 +184,12 @@ def test_host_validation(L):
     assert L.rf2_block_sparse_attn(G(bad_dim), fake, fake, fake, fake, fake, fake, fake, None, None) == \
         rf2.RF2_ERR_UNSUPPORTED
     assert L.rf2_permutation_index(G(good), None) == rf2.RF2_ERR_INVALID_ARGUMENT
+
+
+def test_selftest_timeout_argument_validation(L):
+    """The timeout self-test rejects a limit outside 1 us .. 1 s before any launch."""
+    import ctypes
+    n = ctypes.c_int32(0)
+    for bad in (0, 1_000_001):
+        assert L.rf2_selftest_wait_timeout(ctypes.c_uint32(bad), ctypes.byref(n), None) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_selftest_wait_timeout(ctypes.c_uint32(1000), None, None) == rf2.RF2_ERR_INVALID_ARGUMENT
