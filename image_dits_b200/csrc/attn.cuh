@@ -14,10 +14,10 @@
 // A step is one union entry (64 keys): S_e = Q K_e^T is an M128 x N64
 // product into one of two 64-column S buffers of TMEM, then O += P_e V_e.
 // With two S buffers the product for entry e+1 runs while the softmax of
-// entry e does, so the softmax warps go from one entry to the next without
-// waiting for the tensor pipe; the N = 64 product runs at 2/3 of the N = 128
-// rate (M128 x N64 x K16: 48 cycles against 64), which the overlap more than
-// repays.
+// entry e does, so the softmax warps find the next scores (nearly) ready
+// instead of waiting for the PV and S products of a single-buffer chain; the
+// N = 64 product runs at 2/3 of the N = 128 rate (M128 x N64 x K16: 48
+// cycles against 64), which the overlap more than repays.
 //
 // Roles (256 threads, two CTAs per SM):
 //   warps 0-3  softmax + epilogue: thread r owns query row r = TMEM lane r
@@ -125,6 +125,7 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], float sl2, fl
     sum4[0] = acc[0].x; sum4[1] = acc[0].y; sum4[2] = acc[1].x; sum4[3] = acc[1].y;
 }
 
+// max(acc, s[0..nvalid)) over one 32-score chunk, four independent chains.
 template <bool kMasked>
 __device__ __forceinline__ float max_chunk(const uint32_t (&s)[32], int nvalid, float acc)
 {
