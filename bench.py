@@ -325,7 +325,14 @@ def main():
     mask, ws = rf2.alloc_mask(g, 1.0 if args.tau is not None else wl.keep, dev)
     stream = torch.cuda.current_stream()
 
-    score_groups = -(-wl.batch * wl.heads // 16)
+    # heads per (scores, select) launch pair, as the library groups them: as many
+    # heads' scores as fit in 96 MiB, at most one score item (head, 128-row tile) per SM
+    Tb_ = wl.num_blocks
+    head_bytes = Tb_ * ((Tb_ + 3) // 4 * 4) * 4
+    tiles = (Tb_ + 127) // 128
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    G = min(wl.batch * wl.heads, max(1, (96 << 20) // head_bytes), max(1, sms // tiles))
+    score_groups = -(-wl.batch * wl.heads // G)
 
     def step(ev=None):
         if ev is not None:
@@ -349,7 +356,7 @@ def main():
         if ev is not None:
             ev[5].record(stream)
 
-    # permute+pool, permute V, (scores + select) per group of 16 heads, attention, unpermute
+    # permute+pool, permute V, (scores + select) per group of heads, attention, unpermute
     launches_per_step = 2 + 2 * score_groups + 2
 
     for _ in range(args.warmup):
