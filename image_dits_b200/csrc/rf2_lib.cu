@@ -22,11 +22,11 @@ namespace rf2 {
 
 // Device status word: kernels OR error bits into it; rf2_device_status
 // reads and clears it.
-#ifndef RF2_SELECT_REG
-#define RF2_SELECT_REG 1
-#endif
-
 __device__ int g_status_word;
+
+// Top-n selection keeps rows of up to this many key blocks in registers
+// (select_probe_kernel, 16 keys per lane); see launch_select_topn.
+constexpr int32_t kSelectRegMaxBlocks = 32 * 16;
 
 constexpr int32_t kMaxBlocks = 4096;     // T_b limit (N <= 262,144 tokens)
 
@@ -323,14 +323,11 @@ static int launch_select_probe(const Checked& c, const MaskGeo& mg, const float*
 static int launch_select_topn(const Checked& c, const MaskGeo& mg, const float* S, int64_t h0, int64_t g,
                               int32_t* row_start, int32_t* row_count, int32_t* col_idx, cudaStream_t s)
 {
-    // Keys in registers pay off while a lane holds few of them (measured:
-    // 11% faster at T_b = 512; at T_b = 1182, 40 keys per lane, the register
-    // footprint halves occupancy and the shared-memory radix select is faster).
     // Keys in registers pay off while a lane holds few of them (measured: the
     // image shape's mask 19% faster, 480p equal; at T_b = 1182, 40 keys per
     // lane, the register footprint halves occupancy and the shared-memory
     // radix select is faster).
-    if (RF2_SELECT_REG && c.Tb <= 32 * 16)
+    if (c.Tb <= kSelectRegMaxBlocks)
         return launch_select_probe<16>(c, mg, S, h0, g, row_start, row_count, col_idx, s);
     return launch_select<8>(c, mg, S, h0, g, row_start, row_count, col_idx, s);
 }
