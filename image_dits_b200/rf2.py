@@ -312,11 +312,13 @@ class HostPipeline:
 
     Build once (device buffers, streams and masks are allocated here), then
     call `run(q, k, v, o)` with pinned host bf16 tensors [B, H, N, d].
-    Selection: top-n with `keep`, or the CDF threshold with `tau`.
+    Selection: top-n with `keep`, or the CDF threshold with `tau`.  The heads
+    are split into `chunks` equal chunks, the last of them (with `tail_split`)
+    further into shrinking parts down to one head.
     """
 
     def __init__(self, geom: Geometry, keep: float | None = None, tau: float | None = None, chunks: int = 8,
-                 device=None):
+                 device=None, tail_split: bool = True):
         if (keep is None) == (tau is None):
             raise ValueError("give exactly one of keep and tau")
         self.geom, self.keep, self.tau = geom, keep, tau
@@ -325,8 +327,22 @@ class HostPipeline:
         BH = geom.batch * geom.heads
         n = max(1, min(int(chunks), BH))
         cuts = [round(c * BH / n) for c in range(n + 1)]
+        sizes = [cuts[c + 1] - cuts[c] for c in range(n)]
+        if tail_split:
+            # The host-to-device copies set the pace; what follows the last of
+            # them is the last chunk's compute and copy back, so the last chunk
+            # is split in shrinking parts down to one head.
+            r, tail = sizes.pop(), []
+            while r > 1:
+                h = (r + 1) // 2
+                tail.append(h)
+                r -= h
+            sizes += tail + ([r] if r else [])
+        cuts = [0]
+        for sz in sizes:
+            cuts.append(cuts[-1] + sz)
         self.parts = []
-        for c in range(n):
+        for c in range(len(sizes)):
             h0, h1 = cuts[c], cuts[c + 1]
             g = make_geometry(1, h1 - h0, geom.head_dim, geom.frames, geom.height, geom.width, geom.win_t,
                               geom.win_h, geom.win_w, geom.first_frame_sink, geom.block, geom.text_tokens)
