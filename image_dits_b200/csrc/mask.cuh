@@ -179,34 +179,18 @@ __device__ __forceinline__ uint32_t float_order_key(float f)
 
 constexpr int kSelThreads = 256;
 
-// Selection of one non-sink or sink row i of head bh from its T_b score keys
-// (order-preserving uint32), by one warp: the n-th largest key by a 4-pass
-// 8-bit radix select (hist: 256 words of this warp's shared memory), then the
-// kept set {key > thr} + the lowest-indexed keys == thr up to n, plus every
-// sink column, written in ascending order at the row's closed-form offset.
-__device__ __forceinline__ void select_row(const uint32_t* rk, uint32_t* hist, const MaskGeo& mg, int64_t bh, int i,
-                                           int lane, int32_t* row_start, int32_t* row_count, int32_t* col_idx,
-                                           bool keep_all)
+// The r-th largest (1 <= r <= cnt) of keys[0..cnt), all of which share the
+// high bits common to kmin and kmax (bounds of the keys, not necessarily
+// attained), by one warp: 8-bit radix digits from just below those common
+// bits (hist: 256 words of this warp's shared memory).  Returns the key;
+// `remaining` receives how many keys equal to it are among the r largest.
+__device__ __forceinline__ uint32_t radix_kth(const uint32_t* keys, int cnt, int r, uint32_t kmin, uint32_t kmax,
+                                              uint32_t* hist, int lane, int& remaining)
 {
-    const int Tb = mg.Tb;
-    const int64_t rs = row_offset(mg, bh, i);
-    const int64_t row_id = bh * Tb + i;
-    int32_t* out = col_idx + rs;
-    if (i >= mg.sink_first || keep_all) {
-        for (int j = lane; j < Tb; j += 32) out[j] = j;
-        if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = Tb; }
-        return;
-    }
-    // Keys of a row often share many leading bits (scores cluster): start the
-    // 8-bit digits just below the bits common to the row's min and max key.
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int j = lane; j < Tb; j += 32) { const uint32_t k = rk[j]; kmin = min(kmin, k); kmax = max(kmax, k); }
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    const int common = __clz(kmin ^ kmax);                  // 32 when every key is equal
+    const int common = __clz(kmin ^ kmax);                  // 32 when kmin == kmax
     uint32_t pmask = (common >= 32) ? 0xffffffffu : ~(0xffffffffu >> common);
     uint32_t prefix = kmax & pmask;
-    int remaining = mg.n_keep;
+    remaining = r;
     const int top = 32 - common;                            // undetermined low bits
     #pragma unroll 1
     for (int lo = top - 8; lo > -8; lo -= 8) {
@@ -217,20 +201,20 @@ __device__ __forceinline__ void select_row(const uint32_t* rk, uint32_t* hist, c
         __syncwarp();
         // Lanes hitting the same bin add once (the scores of a row are
         // concentrated, so a warp's 32 keys often share one or two bins).
-        for (int j0 = 0; j0 < Tb; j0 += 32) {
+        for (int j0 = 0; j0 < cnt; j0 += 32) {
             const int j = j0 + lane;
-            const uint32_t k = (j < Tb) ? rk[j] : 0u;
-            const bool hit = (j < Tb) && ((k & pmask) == prefix);
+            const uint32_t k = (j < cnt) ? keys[j] : 0u;
+            const bool hit = (j < cnt) && ((k & pmask) == prefix);
             const uint32_t bin = hit ? ((k >> shift) & 255u) : 256u;
             const uint32_t peers = __match_any_sync(0xffffffffu, bin);
             if (hit && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
         }
         __syncwarp();
         // Lane l owns bins 255-8l .. 248-8l (descending).
-        uint32_t cnt[8];
+        uint32_t cnt8[8];
         uint32_t local = 0;
         #pragma unroll
-        for (int b = 0; b < 8; ++b) { cnt[b] = hist[255 - (lane * 8 + b)]; local += cnt[b]; }
+        for (int b = 0; b < 8; ++b) { cnt8[b] = hist[255 - (lane * 8 + b)]; local += cnt8[b]; }
         uint32_t incl = local;
         #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -246,8 +230,8 @@ __device__ __forceinline__ void select_row(const uint32_t* rk, uint32_t* hist, c
             uint32_t run = excl;
             #pragma unroll
             for (int b = 0; b < 8; ++b) {
-                if (run + cnt[b] >= (uint32_t)remaining) { bin = 255 - (lane * 8 + b); before = run; break; }
-                run += cnt[b];
+                if (run + cnt8[b] >= (uint32_t)remaining) { bin = 255 - (lane * 8 + b); before = run; break; }
+                run += cnt8[b];
             }
         }
         bin = __shfl_sync(0xffffffffu, bin, src_lane);
@@ -257,10 +241,19 @@ __device__ __forceinline__ void select_row(const uint32_t* rk, uint32_t* hist, c
         pmask |= 255u << shift;
         __syncwarp();
     }
-    // prefix is the threshold key; `remaining` keys equal to it are kept,
-    // the lowest-indexed ones first.
-    const uint32_t thr = prefix;
-    int eq_left = remaining;
+    return prefix;
+}
+
+// Writes row i: the keys above thr, the lowest-indexed `eq_left` keys equal to
+// it, and every sink column, in ascending order at the row's closed-form offset.
+__device__ __forceinline__ void write_row(const uint32_t* rk, const MaskGeo& mg, int64_t bh, int i, int lane,
+                                          uint32_t thr, int eq_left, int32_t* row_start, int32_t* row_count,
+                                          int32_t* col_idx)
+{
+    const int Tb = mg.Tb;
+    const int64_t rs = row_offset(mg, bh, i);
+    const int64_t row_id = bh * Tb + i;
+    int32_t* out = col_idx + rs;
     int written = 0;
     for (int j0 = 0; j0 < Tb; j0 += 32) {
         const int j = j0 + lane;
@@ -275,6 +268,115 @@ __device__ __forceinline__ void select_row(const uint32_t* rk, uint32_t* hist, c
         written += __popc(sel_ballot);
     }
     if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = written; }
+}
+
+// Selection of one non-sink or sink row i of head bh from its T_b score keys
+// (order-preserving uint32), by one warp: the n-th largest key by radix_kth
+// over the whole row (its digits start below the bits common to the row's
+// min and max key), then write_row.  Sink rows (and keep = 1) keep every
+// column.
+__device__ __forceinline__ void select_row(const uint32_t* rk, uint32_t* hist, const MaskGeo& mg, int64_t bh, int i,
+                                           int lane, int32_t* row_start, int32_t* row_count, int32_t* col_idx,
+                                           bool keep_all)
+{
+    const int Tb = mg.Tb;
+    if (i >= mg.sink_first || keep_all) {
+        const int64_t rs = row_offset(mg, bh, i);
+        const int64_t row_id = bh * Tb + i;
+        int32_t* out = col_idx + rs;
+        for (int j = lane; j < Tb; j += 32) out[j] = j;
+        if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = Tb; }
+        return;
+    }
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int j = lane; j < Tb; j += 32) { const uint32_t k = rk[j]; kmin = min(kmin, k); kmax = max(kmax, k); }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    int remaining;
+    const uint32_t thr = radix_kth(rk, Tb, mg.n_keep, kmin, kmax, hist, lane, remaining);
+    write_row(rk, mg, bh, i, lane, thr, remaining, row_start, row_count, col_idx);
+}
+
+#ifndef RF2_SELECT_SAMPLED
+#define RF2_SELECT_SAMPLED 1
+#endif
+constexpr int kSelCand = 512;                               // candidate keys per warp (words)
+
+// Top-n of a long row from a sample (same threshold and ties as select_row):
+// 64 keys, one from each of 64 equal stripes of the row, are sorted (warp bitonic sort, two per
+// lane); the n-th largest key is bracketed between the sample keys ranked
+// pos - 8 and pos + 8 (pos = its expected rank in the sample: about 2.5
+// standard deviations of a sample quantile either side); one pass counts the
+// keys above the bracket and gathers the keys inside it, and radix_kth ranks
+// the gathered keys.  When the bracket misses the n-th key or holds more than
+// kSelCand keys, the row goes through select_row.
+__device__ __forceinline__ void select_row_sampled(const uint32_t* rk, uint32_t* hist, uint32_t* cand,
+                                                   const MaskGeo& mg, int64_t bh, int i, int lane,
+                                                   int32_t* row_start, int32_t* row_count, int32_t* col_idx,
+                                                   bool keep_all)
+{
+    const int Tb = mg.Tb, n = mg.n_keep;
+    if (i >= mg.sink_first || keep_all || Tb < 256) {
+        select_row(rk, hist, mg, bh, i, lane, row_start, row_count, col_idx, keep_all);
+        return;
+    }
+    // sample e = 2*lane + s: one position in stripe e of the row's 64 equal
+    // stripes, at an offset drawn from (row, e) (stratified sampling: a fixed
+    // stride follows the scores' smooth structure and biases the quantile);
+    // then sorted descending in e
+    auto pick = [&](int e) -> int {
+        const int s0 = (e * Tb) >> 6, s1 = ((e + 1) * Tb) >> 6;          // stripe [s0, s1), s1 > s0
+        const uint32_t h = (uint32_t)(i * 0x9E3779B1u) ^ (uint32_t)(e * 0x85EBCA77u);
+        return s0 + (int)((h ^ (h >> 15)) % (uint32_t)(s1 - s0));
+    };
+    uint32_t v0 = rk[pick(2 * lane)], v1 = rk[pick(2 * lane + 1)];
+    #pragma unroll
+    for (int k = 2; k <= 64; k <<= 1) {
+        #pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const bool desc = ((2 * lane) & k) == 0;          // same for both elements of the lane
+            if (j == 1) {
+                const uint32_t a = max(v0, v1), b = min(v0, v1);
+                v0 = desc ? a : b;
+                v1 = desc ? b : a;
+            } else {
+                const uint32_t o0 = __shfl_xor_sync(0xffffffffu, v0, j >> 1);
+                const uint32_t o1 = __shfl_xor_sync(0xffffffffu, v1, j >> 1);
+                const bool keep_max = (((2 * lane) & j) == 0) == desc;
+                v0 = keep_max ? max(v0, o0) : min(v0, o0);
+                v1 = keep_max ? max(v1, o1) : min(v1, o1);
+            }
+        }
+    }
+    auto sample_at = [&](int e) -> uint32_t {
+        const uint32_t a = __shfl_sync(0xffffffffu, v0, e >> 1);
+        const uint32_t b = __shfl_sync(0xffffffffu, v1, e >> 1);
+        return (e & 1) ? b : a;
+    };
+    const int pos = (int)(((int64_t)n * 64) / Tb);
+    const uint32_t hi = sample_at(max(0, pos - 8));
+    const uint32_t lo = sample_at(min(63, pos + 8));       // lo <= hi
+    int c_gt = 0, c_in = 0;
+    for (int j0 = 0; j0 < Tb; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t k = (j < Tb) ? rk[j] : 0u;
+        const bool gt = (j < Tb) && k > hi;
+        const bool in = (j < Tb) && k <= hi && k >= lo;
+        const uint32_t bi = __ballot_sync(0xffffffffu, in);
+        const int at = c_in + __popc(bi & ((1u << lane) - 1u));
+        if (in && at < kSelCand) cand[at] = k;
+        c_gt += __popc(__ballot_sync(0xffffffffu, gt));
+        c_in += __popc(bi);
+    }
+    __syncwarp();
+    if (!(c_gt < n && n <= c_gt + c_in && c_in <= kSelCand)) {
+        select_row(rk, hist, mg, bh, i, lane, row_start, row_count, col_idx, keep_all);
+        return;
+    }
+    int remaining;
+    const uint32_t thr = radix_kth(cand, c_in, n - c_gt, lo, hi, hist, lane, remaining);
+    write_row(rk, mg, bh, i, lane, thr, remaining, row_start, row_count, col_idx);
+    __syncwarp();
 }
 
 // ------------------------------------------------------------------------
@@ -485,7 +587,7 @@ __global__ void __launch_bounds__(kSelThreads) select_from_scores_kernel(const f
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int Tb = mg.Tb;
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw);            // [R][Tb]
-    uint32_t* hist_all = keys + (size_t)R * Tb;                          // [8][256]
+    uint32_t* hist_all = keys + (size_t)R * Tb;                          // [8][256], then [8][kSelCand]
     const int64_t hl = blockIdx.y;                                        // head within the group
     const int64_t bh = h0 + hl;
     const int i0 = blockIdx.x * R;
@@ -495,14 +597,29 @@ __global__ void __launch_bounds__(kSelThreads) select_from_scores_kernel(const f
     const int warp = tid >> 5;
     const bool keep_all = mg.n_keep >= Tb;
     const int n_score_rows = keep_all ? 0 : max(0, min(nrows, mg.sink_first - i0));
-    for (int r = 0; r < n_score_rows; ++r) {
-        const float* src = S + (hl * Tb + i0 + r) * (int64_t)ld_s;
-        for (int j = tid; j < Tb; j += kSelThreads) keys[(size_t)r * Tb + j] = float_order_key(src[j]);
+    // the rows' scores as keys: 16-byte loads (rows are ld_s = T_b rounded up
+    // to 4 floats apart), all rows of the CTA in flight together
+    const int nq = (Tb + 3) >> 2;
+    for (int idx = tid; idx < n_score_rows * nq; idx += kSelThreads) {
+        const int r = idx / nq, q4 = idx - r * nq;
+        const float4 f = *reinterpret_cast<const float4*>(S + (hl * Tb + i0 + r) * (int64_t)ld_s + 4 * q4);
+        uint32_t* dst = keys + (size_t)r * Tb + 4 * q4;
+        const int j = 4 * q4;
+        dst[0] = float_order_key(f.x);
+        if (j + 1 < Tb) dst[1] = float_order_key(f.y);
+        if (j + 2 < Tb) dst[2] = float_order_key(f.z);
+        if (j + 3 < Tb) dst[3] = float_order_key(f.w);
     }
     __syncthreads();
     uint32_t* hist = hist_all + warp * 256;
-    for (int r = warp; r < nrows; r += kSelThreads / 32)
-        select_row(keys + (size_t)r * Tb, hist, mg, bh, i0 + r, lane, row_start, row_count, col_idx, keep_all);
+    uint32_t* cand = hist_all + (kSelThreads / 32) * 256 + warp * kSelCand;
+    for (int r = warp; r < nrows; r += kSelThreads / 32) {
+        if (RF2_SELECT_SAMPLED)
+            select_row_sampled(keys + (size_t)r * Tb, hist, cand, mg, bh, i0 + r, lane, row_start, row_count, col_idx,
+                               keep_all);
+        else
+            select_row(keys + (size_t)r * Tb, hist, mg, bh, i0 + r, lane, row_start, row_count, col_idx, keep_all);
+    }
 }
 
 // Inverse of float_order_key.

@@ -300,7 +300,7 @@ template <int R>
 static int launch_select(const Checked& c, const MaskGeo& mg, const float* S, int64_t h0, int64_t g,
                          int32_t* row_start, int32_t* row_count, int32_t* col_idx, cudaStream_t s)
 {
-    const size_t smem = sizeof(uint32_t) * ((size_t)R * c.Tb + 256 * (kSelThreads / 32));
+    const size_t smem = sizeof(uint32_t) * ((size_t)R * c.Tb + (256 + kSelCand) * (kSelThreads / 32));
     if (cudaFuncSetAttribute(select_from_scores_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return RF2_ERR_CUDA;
