@@ -21,6 +21,7 @@ collective on the data path); the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -285,6 +286,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="video720p", choices=list(WORKLOADS))
     ap.add_argument("--keep", type=float, default=None)
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (smaller cases of the same shape, e.g. for ncu)")
     ap.add_argument("--tau", type=float, default=None,
                     help="CDF-threshold selection with this tau instead of the workload's top-n keep ratio")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -300,6 +303,10 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.keep is not None:
         wl = wl.with_keep(args.keep)
+    if args.heads is not None:
+        if args.heads < 1:
+            raise SystemExit("--heads must be >= 1")
+        wl = dataclasses.replace(wl, heads=args.heads, name=f"{wl.name}@heads{args.heads}")
 
     if args.impl == "reference":
         run_reference(args, wl, rank)
