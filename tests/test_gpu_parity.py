@@ -238,6 +238,25 @@ def test_random_geometries():
         assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, (wl, e)
 
 
+@pytest.mark.parametrize("keep,sink", [(0.02, True), (0.2, False), (0.6, True), (0.97, False)])
+def test_long_rows_selection(keep, sink):
+    """Rows of more than 512 key blocks take the shared-memory selection (a
+    stratified sample brackets the n-th largest score, a radix select ranks
+    the bracketed keys, the whole row where the bracket misses): masks match
+    the oracle at small and large keep ratios (the bracket clamped at either
+    end of the sample), with and without the first-frame sink."""
+    wl = Workload("long", 1, 2, 64, 4, 64, 144, 2, 8, 8, keep, sink, (24, 20, 20))
+    assert wl.num_blocks > 512
+    q, k, v = make_qkv(wl, "cuda", seed=31)
+    g = rf2.geometry_of(wl)
+    qp, kp = rf2.permute(g, q), rf2.permute(g, k)
+    mask = rf2.predict_mask(g, qp, kp, keep)
+    torch.cuda.synchronize()
+    assert rf2.device_status() == rf2.RF2_OK
+    check_csr(mask, mask.sizes.sink_first)
+    compare_masks(mask.dense(), bits(qp), bits(kp), keep, wl.frames, wl.height, wl.width, sink)
+
+
 def _full_size(name, n_random_blocks, n_sink_blocks):
     wl = WORKLOADS[name]
     q, k, v = make_qkv(wl, "cuda", seed=0)
