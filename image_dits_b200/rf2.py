@@ -300,6 +300,24 @@ def rainfusion_attention(geom: Geometry, q, k, v, keep: float, stream=None):
     return unpermute(geom, op, stream=stream), mask
 
 
+def chunk_sizes(heads: int, chunks: int, tail_split: bool = True) -> list:
+    """Heads per chunk of a HostPipeline: `chunks` near-equal chunks; with
+    `tail_split` the last one is further split in shrinking parts down to one
+    head (the host-to-device copies set the pace, and what follows the last of
+    them is the last chunk's compute and copy back)."""
+    n = max(1, min(int(chunks), int(heads)))
+    cuts = [round(c * heads / n) for c in range(n + 1)]
+    sizes = [cuts[c + 1] - cuts[c] for c in range(n)]
+    if tail_split:
+        r, tail = sizes.pop(), []
+        while r > 1:
+            h = (r + 1) // 2
+            tail.append(h)
+            r -= h
+        sizes += tail + ([r] if r else [])
+    return sizes
+
+
 class HostPipeline:
     """One attention call on host (pinned) tensors, copies overlapped with compute.
 
@@ -325,19 +343,7 @@ class HostPipeline:
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         self.device = dev
         BH = geom.batch * geom.heads
-        n = max(1, min(int(chunks), BH))
-        cuts = [round(c * BH / n) for c in range(n + 1)]
-        sizes = [cuts[c + 1] - cuts[c] for c in range(n)]
-        if tail_split:
-            # The host-to-device copies set the pace; what follows the last of
-            # them is the last chunk's compute and copy back, so the last chunk
-            # is split in shrinking parts down to one head.
-            r, tail = sizes.pop(), []
-            while r > 1:
-                h = (r + 1) // 2
-                tail.append(h)
-                r -= h
-            sizes += tail + ([r] if r else [])
+        sizes = chunk_sizes(BH, chunks, tail_split)
         cuts = [0]
         for sz in sizes:
             cuts.append(cuts[-1] + sz)

@@ -193,3 +193,22 @@ def test_selftest_timeout_argument_validation(L):
     for bad in (0, 1_000_001):
         assert L.rf2_selftest_wait_timeout(ctypes.c_uint32(bad), ctypes.byref(n), None) == rf2.RF2_ERR_INVALID_ARGUMENT
     assert L.rf2_selftest_wait_timeout(ctypes.c_uint32(1000), None, None) == rf2.RF2_ERR_INVALID_ARGUMENT
+
+
+def test_host_pipeline_chunk_sizes():
+    """Head chunks of rf2.HostPipeline: every head exactly once, in order; equal
+    chunks (within one head) without the tail split; with it the last equal
+    chunk is split in shrinking parts that end with a single head."""
+    for heads in (1, 2, 3, 7, 12, 24, 40, 97):
+        for chunks in (1, 2, 3, 5, 8, 10, 200):
+            even = rf2.chunk_sizes(heads, chunks, tail_split=False)
+            assert sum(even) == heads and all(s >= 1 for s in even)
+            assert max(even) - min(even) <= 1
+            assert len(even) == min(chunks, heads)
+            split = rf2.chunk_sizes(heads, chunks, tail_split=True)
+            assert sum(split) == heads and all(s >= 1 for s in split)
+            assert split[:len(even) - 1] == even[:-1]
+            tail = split[len(even) - 1:]
+            assert sum(tail) == even[-1] and tail[-1] == 1
+            assert all(a >= b for a, b in zip(tail, tail[1:]))
+    assert rf2.chunk_sizes(40, 8) == [5, 5, 5, 5, 5, 5, 5, 3, 1, 1]
