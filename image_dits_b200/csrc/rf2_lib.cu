@@ -118,10 +118,76 @@ static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg
     return RF2_OK;
 }
 
+// Launch errors are reported per call: every launch helper drops a pending
+// (non-sticky) error left by unrelated earlier work before it launches, and
+// reads and clears its own launch's error after.  A sticky error (a context
+// that has already faulted) persists and is reported by every later call.
+static void clear_pending_error() { (void)cudaGetLastError(); }
+
 static int launch_status()
 {
-    const cudaError_t e = cudaPeekAtLastError();
+    const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? RF2_OK : RF2_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- contexts
+// Per-context caches (the dynamic shared-memory attribute of a kernel) are
+// keyed by the unique id of the calling thread's current CUDA context, so a
+// context created anew (after cudaDeviceReset, say) is set up again instead
+// of trusting state that belonged to the old one.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+static Fn driver_fn(const char* name)
+{
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<Fn>(p);
+    return nullptr;
+}
+
+// Unique id of the current context; false when there is none or it cannot be read.
+static bool current_context_id(unsigned long long* id)
+{
+    static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (!get_current || !get_id) return false;
+    CUcontext c = nullptr;
+    if (get_current(&c) != CUDA_SUCCESS || !c) return false;
+    return get_id(c, id) == CUDA_SUCCESS;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, context),
+// raised when a later call needs more.
+static int ensure_dynamic_smem(const void* func, size_t bytes)
+{
+    struct Entry { const void* func; unsigned long long ctx; size_t bytes; };
+    static Entry cache[64];
+    static int used = 0;
+    static std::mutex mu;
+    unsigned long long ctx = 0;
+    const bool have_ctx = current_context_id(&ctx);
+    std::lock_guard<std::mutex> lock(mu);
+    Entry* e = nullptr;
+    if (have_ctx)
+        for (int i = 0; i < used; ++i)
+            if (cache[i].func == func && cache[i].ctx == ctx) { e = &cache[i]; break; }
+    if (e && e->bytes >= bytes) return RF2_OK;
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) {
+        clear_pending_error();
+        return RF2_ERR_CUDA;
+    }
+    if (!have_ctx) return RF2_OK;
+    if (!e) {
+        e = &cache[used < 64 ? used++ : (int)(ctx % 64)];   // full: overwrite a slot (it is set again when needed)
+        e->func = func;
+        e->ctx = ctx;
+        e->bytes = 0;
+    }
+    e->bytes = bytes;
+    return RF2_OK;
 }
 
 static int grid_for_rows(int64_t rows)
@@ -147,6 +213,7 @@ static int permute_impl(const rf2_geometry* geom, const void* in, void* out, voi
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const uint4* i4 = reinterpret_cast<const uint4*>(in);
     uint4* o4 = reinterpret_cast<uint4*>(out);
+    clear_pending_error();
     if (c.D == 128) {
         if (forward) permute_rows_kernel<128, true><<<grid, 256, 0, s>>>(i4, o4, c.pg, rows);
         else         permute_rows_kernel<128, false><<<grid, 256, 0, s>>>(i4, o4, c.pg, rows);
@@ -242,10 +309,10 @@ static int launch_attn(const Checked& c, const MaskGeo& mg, const void* qp, cons
     a.sink_pairs = (mg.sink_first < c.Tb) ? a.pairs - mg.sink_first / 2 : 0;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     const size_t smem = Cfg::smem_bytes(c.Tb);
-    if (cudaFuncSetAttribute(block_sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (ensure_dynamic_smem(reinterpret_cast<const void*>(block_sparse_attn_kernel<D>), smem) != RF2_OK)
         return RF2_ERR_CUDA;
     const int64_t grid = c.BH * a.pairs;
+    clear_pending_error();
     block_sparse_attn_kernel<D><<<(unsigned)grid, Cfg::THREADS, smem, s>>>(mq, mk, mv, a);
     return launch_status();
 }
@@ -286,11 +353,11 @@ static int launch_scores(const Checked& c, const float* means_hi, const float* m
     if (!make_means_map(&mh, means_hi, D, rows, 128) || !make_means_map(&ml, means_lo, D, rows, 128) ||
         !make_means_map(&mhb, means_hi, D, rows, Cfg::NCH) || !make_means_map(&mlb, means_lo, D, rows, Cfg::NCH))
         return RF2_ERR_CUDA;
-    if (cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) !=
-        cudaSuccess)
+    if (ensure_dynamic_smem(reinterpret_cast<const void*>(score_tc_kernel<D>), Cfg::SMEM) != RF2_OK)
         return RF2_ERR_CUDA;
     const int64_t items = g * ((c.Tb + 127) / 128);
     const int grid = (int)(items < num_sms() ? items : num_sms());
+    clear_pending_error();
     score_tc_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM, s>>>(mh, ml, mhb, mlb, S, c.Tb, score_ld(c.Tb), c.BH, h0,
                                                              (int32_t)g, (float)(1.0 / sqrt((double)D)), status);
     return launch_status();
@@ -301,10 +368,10 @@ static int launch_select(const Checked& c, const MaskGeo& mg, const float* S, in
                          int32_t* row_start, int32_t* row_count, int32_t* col_idx, cudaStream_t s)
 {
     const size_t smem = sizeof(uint32_t) * ((size_t)R * c.Tb + (256 + kSelCand) * (kSelThreads / 32));
-    if (cudaFuncSetAttribute(select_from_scores_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (ensure_dynamic_smem(reinterpret_cast<const void*>(select_from_scores_kernel<R>), smem) != RF2_OK)
         return RF2_ERR_CUDA;
     dim3 grid((c.Tb + R - 1) / R, (unsigned)g);
+    clear_pending_error();
     select_from_scores_kernel<R><<<grid, kSelThreads, smem, s>>>(S, score_ld(c.Tb), row_start, row_count,
                                                                  col_idx, mg, h0);
     return launch_status();
@@ -316,6 +383,7 @@ static int launch_select_probe(const Checked& c, const MaskGeo& mg, const float*
 {
     constexpr int rows_per_cta = kSelThreads / 32;
     dim3 grid((c.Tb + rows_per_cta - 1) / rows_per_cta, (unsigned)g);
+    clear_pending_error();
     select_probe_kernel<KPL><<<grid, kSelThreads, 0, s>>>(S, score_ld(c.Tb), row_start, row_count, col_idx, mg, h0);
     return launch_status();
 }
@@ -339,10 +407,10 @@ static int launch_select_cdf(const Checked& c, const MaskGeo& mg, const float* S
                              int32_t* row_start, int32_t* row_count, int32_t* col_idx, float tau, cudaStream_t s)
 {
     const size_t smem = (size_t)R * c.Tb * 8;
-    if (cudaFuncSetAttribute(select_cdf_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+    if (ensure_dynamic_smem(reinterpret_cast<const void*>(select_cdf_kernel<R>), smem) != RF2_OK)
         return RF2_ERR_CUDA;
     dim3 grid((c.Tb + R - 1) / R, (unsigned)g);
+    clear_pending_error();
     select_cdf_kernel<R><<<grid, 32 * R, smem, s>>>(S, score_ld(c.Tb), row_start, row_count, col_idx, mg, h0, tau);
     return launch_status();
 }
@@ -408,6 +476,7 @@ static int launch_mask(const Checked& c, const MaskGeo& mg, const void* qp, cons
     if (st != RF2_OK) return st;
     const int64_t warps = 2 * c.BH * c.Tb;
     const unsigned grid = (unsigned)((warps + 7) / 8);
+    clear_pending_error();
     if (c.D == 128)
         block_mean_kernel<128><<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(qp),
                                                      reinterpret_cast<const uint4*>(kp), w.means_hi, w.means_lo,
@@ -425,26 +494,20 @@ static int launch_mask(const Checked& c, const MaskGeo& mg, const void* qp, cons
 // Fixed device scratch for rf2_predict_mask_static (callers that cannot
 // allocate).  Every device that loads this library holds these 64 MiB until
 // the process exits.  In host code `g_static_scratch` only names a host-side
-// stand-in, so its device address is looked up once per device.
+// stand-in, so every call looks up its device address on the current device
+// (no cached pointer can outlive the context it was read in).
 constexpr size_t kStaticScratchBytes = (size_t)64 << 20;
 static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
 
-constexpr int kMaxDevices = 64;
-static float* g_static_scratch_addr[kMaxDevices];
-static std::mutex g_static_scratch_mutex;
-
-// Device address of the scratch on the current device (set-up on first use).
+// Device address of the scratch on the calling thread's current device.
 static int static_scratch(float** out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RF2_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
-    if (!g_static_scratch_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return RF2_ERR_CUDA;
-        g_static_scratch_addr[dev] = static_cast<float*>(p);
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+        clear_pending_error();
+        return RF2_ERR_CUDA;
     }
-    *out = g_static_scratch_addr[dev];
+    *out = static_cast<float*>(p);
     return RF2_OK;
 }
 
@@ -571,6 +634,7 @@ int rf2_permute_qk_pool(const rf2_geometry* geom, const void* q, const void* k, 
     int64_t grid = (blocks + 7) / 8;
     const int64_t cap = (int64_t)num_sms() * 16;
     if (grid > cap) grid = cap;
+    clear_pending_error();
     if (c.D == 128)
         permute_pool_kernel<128><<<(unsigned)grid, 256, 0, s>>>(
             reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), reinterpret_cast<uint4*>(qp),
@@ -680,6 +744,7 @@ int rf2_selftest_wait_timeout(uint32_t limit_us, int32_t* waits_given_up, void* 
     int* status = status_word_ptr();
     int* left = selftest_counter();
     if (!status || !left) return RF2_ERR_CUDA;
+    clear_pending_error();
     if (cudaMemsetAsync(left, 0, sizeof(int), s) != cudaSuccess) return RF2_ERR_CUDA;
     selftest_timeout_kernel<<<1, 64, 0, s>>>((uint64_t)limit_us * 1000u, status, left);
     const int r = launch_status();

@@ -24,7 +24,9 @@
  *   Every call is asynchronous on it and launches 1-2 kernels.
  * - Arguments are validated on the host before anything is launched; an
  *   invalid call returns an error status and launches nothing.  A failed
- *   launch returns RF2_ERR_CUDA.  Kernels never trap: a bounded wait that
+ *   launch returns RF2_ERR_CUDA (a pending error left by unrelated earlier
+ *   work is cleared before the call launches, so it is not reported as this
+ *   call's; an error that has made the context unusable is).  Kernels never trap: a bounded wait that
  *   runs out records RF2_ERR_TIMEOUT in a device status word that
  *   rf2_device_status reads back.
  * - Blocks are 64 consecutive tokens of the permuted sequence; T_b =
@@ -141,9 +143,11 @@ int rf2_predict_mask(const rf2_geometry* geom, const void* qp_bf16, const void* 
  *   larger problems return RF2_ERR_INSUFFICIENT_WORKSPACE and launch nothing
  *   (split the heads over several calls, or use rf2_predict_mask).
  * - Every GPU that loads the library holds the 64 MiB until the process exits.
- * - The first call on a device looks up the array's device address (with that
- *   device current) and caches it; make that first call before any stream
- *   capture.  It allocates nothing, and calls no allocating routine.
+ * - Every call looks up the array's device address on the calling thread's
+ *   current device (cudaGetSymbolAddress; nothing is cached, so a context
+ *   created anew after cudaDeviceReset is served correctly).  The first call
+ *   on a device also loads the library's device code there: make it before
+ *   any stream capture.  No call allocates, or calls an allocating routine.
  * - All calls share the one array and it keeps the last call's contents;
  *   nothing in it needs to start at zero, but calls that overlap on the GPU
  *   (different streams, or different host threads on one device) race on it.

@@ -212,3 +212,20 @@ def test_host_pipeline_chunk_sizes():
             assert sum(tail) == even[-1] and tail[-1] == 1
             assert all(a >= b for a, b in zip(tail, tail[1:]))
     assert rf2.chunk_sizes(40, 8) == [5, 5, 5, 5, 5, 5, 5, 3, 1, 1]
+
+
+def test_static_scratch_size_limit_on_host(L):
+    """rf2_predict_mask_static refuses, on the host and before any device call,
+    a problem whose block means (hi/lo pair) plus one head's pooled scores
+    exceed its 64 MiB array: at 720p that is 26 heads and more (25 fit)."""
+    import dataclasses
+    fake = ctypes.c_void_p(0x10000)
+    for heads, fits in ((25, True), (26, False), (40, False)):
+        g = rf2.geometry_of(dataclasses.replace(WORKLOADS["video720p"], heads=heads))
+        Tb = 1182
+        means = (2 * heads * Tb * 128 * 4 + 255) // 256 * 256
+        need = 2 * means + Tb * ((Tb + 3) // 4 * 4) * 4
+        assert (need <= 64 << 20) == fits
+        if not fits:
+            st = L.rf2_predict_mask_static(ctypes.byref(g), fake, fake, 0.2, fake, fake, fake, None)
+            assert st == rf2.RF2_ERR_INSUFFICIENT_WORKSPACE

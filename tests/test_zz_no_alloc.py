@@ -59,11 +59,35 @@ def test_static_scratch_matches_workspace_variant():
         _same(got, ref)
 
 
-def test_static_scratch_refuses_oversize():
+def test_static_scratch_largest_720p_problem():
+    """At 720p (75,600 tokens, d = 128) the scratch holds the block means of
+    25 heads (2 x 30.3 MB as a hi/lo pair) plus one head's pooled scores
+    (5.6 MB): 25 heads, the documented limit, run and match rf2_predict_mask
+    exactly."""
     rf2_build.build()
-    wl = WORKLOADS["video720p"]
-    g = rf2.geometry_of(wl, batch=2)          # 2 x 40 heads: 96.8 MB of block means > 64 MiB
-    assert rf2.query(g, wl.keep).mask_workspace_bytes > 64 << 20
+    import dataclasses
+    wl = dataclasses.replace(WORKLOADS["video720p"], heads=25)
+    q, k, _ = make_qkv(wl, "cuda", seed=3)
+    g = rf2.geometry_of(wl)
+    qp, kp = rf2.permute(g, q), rf2.permute(g, k)
+    del q, k
+    ref = rf2.predict_mask(g, qp, kp, wl.keep)
+    for _ in range(2):
+        got = _static_mask(g, qp, kp, wl.keep)
+        torch.cuda.synchronize()
+        assert rf2.device_status() == rf2.RF2_OK
+        _same(got, ref)
+
+
+def test_static_scratch_refuses_oversize():
+    """Problems whose block means and one head's scores exceed the 64 MiB
+    array are refused before anything is launched: 26 heads at 720p (2 x
+    31.5 MB of means + 5.6 MB of scores) and 2 x 40 heads (2 x 96.8 MB of
+    means)."""
+    rf2_build.build()
+    import dataclasses
     fake = ctypes.c_void_p(0x10000)            # never touched: the size check comes first
-    st = rf2.lib().rf2_predict_mask_static(ctypes.byref(g), fake, fake, wl.keep, fake, fake, fake, None)
-    assert st == rf2.RF2_ERR_INSUFFICIENT_WORKSPACE
+    for g in (rf2.geometry_of(dataclasses.replace(WORKLOADS["video720p"], heads=26)),
+              rf2.geometry_of(WORKLOADS["video720p"], batch=2)):
+        st = rf2.lib().rf2_predict_mask_static(ctypes.byref(g), fake, fake, 0.2, fake, fake, fake, None)
+        assert st == rf2.RF2_ERR_INSUFFICIENT_WORKSPACE
