@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librf2.so")
 SOURCES = ["rf2_lib.cu"]
-DEPS = ["rf2_lib.cu", "attn.cuh", "mask.cuh", "permute.cuh", "geometry.cuh", "ptx.cuh"]
+DEPS = ["rf2_lib.cu", "attn.cuh", "mask.cuh", "topn.cuh", "permute.cuh", "geometry.cuh", "ptx.cuh"]
 
 
 def nvcc_cmd(out: str, extra=()) -> list:

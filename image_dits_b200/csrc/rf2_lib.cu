@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -17,6 +18,7 @@
 #include "mask.cuh"
 #include "permute.cuh"
 #include "ptx.cuh"
+#include "topn.cuh"
 
 namespace rf2 {
 
@@ -94,6 +96,25 @@ static int64_t score_group_heads(const Checked& c)
     if (g < 1) g = 1;
     return c.BH < g ? c.BH : g;
 }
+// Top-n selection from codes (topn_codes_kernel, topn_rows_kernel, topn_overflow_kernel): the
+// codes, the per-row histograms and code widths.  They share the region after
+// the means with the score buffer of the score-matrix path (never both in one
+// call); the region is the larger of the two.
+static int64_t topn_items(const Checked& c) { return c.BH * ((c.Tb + 127) / 128); }
+static size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+static size_t codes_bytes(const Checked& c) { return round256(4 * topn_codes_words(topn_items(c), c.Tb)); }
+static size_t hist_bytes(const Checked& c) { return round256(4 * topn_hist_words(topn_items(c))); }
+static size_t width_bytes(const Checked& c) { return round256((size_t)4 * topn_items(c) * 128); }
+static size_t topn_overflow_bytes(const Checked& c) { return round256(4 * topn_overflow_words(c.BH * c.Tb)); }
+static size_t topn_region_bytes(const Checked& c)
+{
+    return 2 * codes_bytes(c) + hist_bytes(c) + width_bytes(c) + topn_overflow_bytes(c);
+}
+static size_t after_means_bytes(const Checked& c, int64_t score_heads)
+{
+    const size_t sb = (size_t)score_heads * score_head_bytes(c), tb = topn_region_bytes(c);
+    return sb > tb ? sb : tb;
+}
 
 static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg, rf2_sizes* out)
 {
@@ -113,7 +134,7 @@ static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg
         out->row_capacity = mg.cap;
         out->num_rows = c.BH * c.Tb;
         out->col_idx_capacity = total;
-        out->mask_workspace_bytes = 2 * mask_means_bytes(c) + (size_t)score_group_heads(c) * score_head_bytes(c);
+        out->mask_workspace_bytes = 2 * mask_means_bytes(c) + after_means_bytes(c, score_group_heads(c));
     }
     return RF2_OK;
 }
@@ -427,10 +448,11 @@ struct MaskWs {
     int64_t G;
 };
 
-static int mask_ws(const Checked& c, void* ws, size_t ws_bytes, MaskWs* w)
+static int mask_ws(const Checked& c, void* ws, size_t ws_bytes, MaskWs* w, bool score_matrix = false)
 {
     const size_t mb = mask_means_bytes(c);
-    if (ws_bytes < 2 * mb + score_head_bytes(c)) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    const size_t need = score_matrix ? score_head_bytes(c) : after_means_bytes(c, 1);
+    if (ws_bytes < 2 * mb + need) return RF2_ERR_INSUFFICIENT_WORKSPACE;
     int64_t G = (int64_t)((ws_bytes - 2 * mb) / score_head_bytes(c));
     if (G > score_group_heads(c)) G = score_group_heads(c);
     // one round of the persistent score kernel: a group's (head, 128-row tile)
@@ -446,11 +468,89 @@ static int mask_ws(const Checked& c, void* ws, size_t ws_bytes, MaskWs* w)
     return RF2_OK;
 }
 
+// Top-n selection without the score matrix: topn_codes_kernel (scores on
+// the tensor cores, reduced to 16-bit codes and per-row histograms as they
+// leave TMEM), topn_rows_kernel (one thread per row) and topn_overflow_kernel
+// (one CTA for each row the former lists).
+template <int D>
+static int launch_topn(const Checked& c, const MaskGeo& mg, const MaskWs& w, int32_t* row_start,
+                       int32_t* row_count, int32_t* col_idx, cudaStream_t s)
+{
+    using Cfg = TopnCfg<D>;
+    int* status = status_word_ptr();
+    if (!status) return RF2_ERR_CUDA;
+    const int64_t rows = 2 * c.BH * c.Tb;
+    CUtensorMap ah, al, bh, bl, rh, rlo;
+    if (!make_means_map(&ah, w.means_hi, D, rows, 128) || !make_means_map(&al, w.means_lo, D, rows, 128) ||
+        !make_means_map(&bh, w.means_hi, D, rows, Cfg::NB) || !make_means_map(&bl, w.means_lo, D, rows, Cfg::NB) ||
+        !make_means_map(&rh, w.means_hi, D, rows, 1) || !make_means_map(&rlo, w.means_lo, D, rows, 1))
+        return RF2_ERR_CUDA;
+    if (ensure_dynamic_smem(reinterpret_cast<const void*>(topn_codes_kernel<D>), Cfg::SMEM) != RF2_OK)
+        return RF2_ERR_CUDA;
+    // topn_rows_kernel: bitmaps [32][G | 1], bin-b* keys [64][32], row kinds [32];
+    // topn_overflow_kernel: the keys of the threshold code, their scores, radix bins
+    const int G = (c.Tb + 31) / 32;
+    const size_t rows_smem = ((size_t)32 * (G | 1) + 64 * 32 + 32) * 4;
+    const size_t ovf_smem = (size_t)(2 * c.Tb + 256) * 4;
+    if (ensure_dynamic_smem(reinterpret_cast<const void*>(topn_rows_kernel<D>), rows_smem) != RF2_OK ||
+        ensure_dynamic_smem(reinterpret_cast<const void*>(topn_overflow_kernel<D>), ovf_smem) != RF2_OK)
+        return RF2_ERR_CUDA;
+    uint8_t* region = reinterpret_cast<uint8_t*>(w.S);
+    TopnArgs a;
+    a.means_hi = w.means_hi;
+    a.means_lo = w.means_lo;
+    a.codes = reinterpret_cast<uint32_t*>(region);
+    a.fine = reinterpret_cast<uint32_t*>(region + codes_bytes(c));
+    a.hist = reinterpret_cast<uint32_t*>(region + 2 * codes_bytes(c));
+    a.width = reinterpret_cast<float*>(region + 2 * codes_bytes(c) + hist_bytes(c));
+    a.overflow = reinterpret_cast<int32_t*>(region + 2 * codes_bytes(c) + hist_bytes(c) + width_bytes(c));
+    a.row_start = row_start;
+    a.row_count = row_count;
+    a.col_idx = col_idx;
+    a.status = status;
+    a.mg = mg;
+    a.BH = c.BH;
+    // Scores are compared unscaled (q^ . k^): 1e-6 after the 1/sqrt(d) scale
+    // is the code width up to which a code's keys count as tied.
+    a.tiny_width = (float)(1e-6 * sqrt((double)D));
+    a.tiny_width_fine = 256.f * a.tiny_width;
+    a.min_width = 120.f * a.tiny_width;
+    const int64_t items = topn_items(c);
+    const int sms = num_sms();
+    const int grid = (int)(items < sms ? items : sms);
+    clear_pending_error();
+    if (cudaMemsetAsync(a.overflow, 0, sizeof(int32_t), s) != cudaSuccess) return RF2_ERR_CUDA;
+    topn_codes_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM, s>>>(ah, al, bh, bl, rh, rlo, a);
+    int r = launch_status();
+    if (r != RF2_OK) return r;
+    const int64_t rows_grid = 4 * items < (int64_t)sms * 12 ? 4 * items : (int64_t)sms * 12;
+    topn_rows_kernel<D><<<(unsigned)rows_grid, 32, rows_smem, s>>>(a);
+    r = launch_status();
+    if (r != RF2_OK) return r;
+    // rows with too many keys near their threshold for topn_rows_kernel (rare; the
+    // launch returns at once when there are none)
+    topn_overflow_kernel<D><<<sms, 256, ovf_smem, s>>>(a);
+    return launch_status();
+}
+
 // Per group of heads: the tensor-core scores, then the selection (top-n, or
 // the CDF threshold when tau > 0).
 static int launch_score_select(const Checked& c, const MaskGeo& mg, const MaskWs& w, int32_t* row_start,
-                               int32_t* row_count, int32_t* col_idx, cudaStream_t s, float tau = 0.f)
+                               int32_t* row_count, int32_t* col_idx, cudaStream_t s, float tau = 0.f,
+                               bool score_matrix = false)
 {
+    // The score-matrix path is the faster one while all heads' scores fit one
+    // group (they then stay in L2); beyond that, selection from codes.  The
+    // environment variable RF2_MASK_SELECT = "codes" or "scores" overrides
+    // the choice (both give the same masks outside the tie band).
+    bool from_codes = (uint64_t)c.BH * score_head_bytes(c) > kScoreGroupBytes;
+    if (const char* e = getenv("RF2_MASK_SELECT")) {
+        if (strcmp(e, "codes") == 0) from_codes = true;
+        else if (strcmp(e, "scores") == 0) from_codes = false;
+    }
+    if (tau <= 0.f && !score_matrix && from_codes && c.Tb <= TopnCfg<128>::MAX_TB)
+        return (c.D == 128) ? launch_topn<128>(c, mg, w, row_start, row_count, col_idx, s)
+                            : launch_topn<64>(c, mg, w, row_start, row_count, col_idx, s);
     int r = RF2_OK;
     for (int64_t h0 = 0; r == RF2_OK && h0 < c.BH; h0 += w.G) {
         const int64_t g = (c.BH - h0 < w.G) ? c.BH - h0 : w.G;
@@ -469,10 +569,10 @@ static int launch_score_select(const Checked& c, const MaskGeo& mg, const MaskWs
 // Block means of the permuted Q and K, then scores and selection.
 static int launch_mask(const Checked& c, const MaskGeo& mg, const void* qp, const void* kp, int32_t* row_start,
                        int32_t* row_count, int32_t* col_idx, void* ws, size_t ws_bytes, cudaStream_t s,
-                       float tau = 0.f)
+                       float tau = 0.f, bool score_matrix = false)
 {
     MaskWs w;
-    const int st = mask_ws(c, ws, ws_bytes, &w);
+    const int st = mask_ws(c, ws, ws_bytes, &w, score_matrix);
     if (st != RF2_OK) return st;
     const int64_t warps = 2 * c.BH * c.Tb;
     const unsigned grid = (unsigned)((warps + 7) / 8);
@@ -487,7 +587,7 @@ static int launch_mask(const Checked& c, const MaskGeo& mg, const void* qp, cons
                                                     c.N, c.Tb, c.BH);
     const int r = launch_status();
     if (r != RF2_OK) return r;
-    return launch_score_select(c, mg, w, row_start, row_count, col_idx, s, tau);
+    return launch_score_select(c, mg, w, row_start, row_count, col_idx, s, tau, score_matrix);
 }
 
 // ------------------------------------------------------------------------
@@ -602,7 +702,9 @@ int rf2_predict_mask_static(const rf2_geometry* geom, const void* qp, const void
     if (!qp || !kp || !row_start || !row_count || !col_idx) return RF2_ERR_INVALID_ARGUMENT;
     if (!aligned16(qp) || !aligned16(kp) || !aligned16(row_start) || !aligned16(row_count) || !aligned16(col_idx))
         return RF2_ERR_INVALID_ARGUMENT;
-    // Needs room for the block means and the scores of at least one head.
+    // Needs room for the block means and the scores of at least one head (the
+    // fixed array serves the score-matrix path: scores and selection head
+    // group by head group, as many heads per group as fit).
     if (2 * mask_means_bytes(c) + score_head_bytes(c) > kStaticScratchBytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
     float* scratch = nullptr;
     const int ss = static_scratch(&scratch);
@@ -610,7 +712,7 @@ int rf2_predict_mask_static(const rf2_geometry* geom, const void* qp, const void
     // Every scratch element the kernels read is written earlier in the same
     // call, so nothing left from an earlier call needs clearing.
     return launch_mask(c, mg, qp, kp, row_start, row_count, col_idx, scratch, kStaticScratchBytes,
-                       reinterpret_cast<cudaStream_t>(stream));
+                       reinterpret_cast<cudaStream_t>(stream), 0.f, true);
 }
 
 int rf2_permute_qk_pool(const rf2_geometry* geom, const void* q, const void* k, void* qp, void* kp,

@@ -85,9 +85,12 @@ typedef struct {
     int64_t num_rows;            /* batch * heads * T_b: length of row_start / row_count */
     int64_t col_idx_capacity;    /* length of col_idx */
     size_t  mask_workspace_bytes;/* scratch for rf2_predict_mask: the block means as a
-                                    tf32 hi/lo pair of fp32 arrays, then the pooled
-                                    scores of as many heads as fit in 96 MiB (at least
-                                    one head; all of them when they fit) */
+                                    tf32 hi/lo pair of fp32 arrays, then the larger of
+                                    (a) the pooled scores of as many heads as fit in
+                                    96 MiB (at least one head; all of them when they
+                                    fit) and (b) two bytes of score code per score,
+                                    per-row code histograms and widths and a row list
+                                    (the top-n path for T_b <= 2048) */
 } rf2_sizes;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -124,12 +127,18 @@ int rf2_unpermute(const rf2_geometry* geom, const void* xp_bf16, void* x_bf16, v
  *   col_idx[row_start[r] .. + row_count[r]) kept key blocks, ascending.
  * row_start/row_count hold num_rows int32, col_idx col_idx_capacity int32,
  * workspace at least mask_workspace_bytes (device, 16-byte aligned); its
- * contents on entry do not matter.  qp/kp are the permuted Q and K. */
+ * contents on entry do not matter.  qp/kp are the permuted Q and K.
+ * Two selections give the same masks outside a 1e-5 band around each row's
+ * threshold: from the score matrix (chosen while the scores of all heads
+ * fit in 96 MiB) and, for larger calls with T_b <= 2048, from 16-bit codes
+ * of the scores that never leave the SM as floats.  The environment
+ * variable RF2_MASK_SELECT = "scores" or "codes" forces one of them (read
+ * on every call; "codes" still needs T_b <= 2048). */
 int rf2_predict_mask(const rf2_geometry* geom, const void* qp_bf16, const void* kp_bf16,
                      double keep_ratio, int32_t* row_start, int32_t* row_count, int32_t* col_idx,
                      void* workspace, size_t workspace_bytes, void* stream);
 
-/* rf2_predict_mask without a caller-supplied workspace: the same computation
+/* rf2_predict_mask without a caller-supplied workspace: the same arguments
  * and outputs, with the block-mean scratch taken from a fixed 64 MiB array
  * inside the library instead.  For callers that cannot allocate device
  * memory themselves — for example code embedded in a host framework that
@@ -142,6 +151,10 @@ int rf2_predict_mask(const rf2_geometry* geom, const void* qp_bf16, const void* 
  *   tokens, d = 128);
  *   larger problems return RF2_ERR_INSUFFICIENT_WORKSPACE and launch nothing
  *   (split the heads over several calls, or use rf2_predict_mask).
+ * - It always selects from the score matrix (rf2_predict_mask with
+ *   RF2_MASK_SELECT=scores gives the identical mask; without it, large calls
+ *   of rf2_predict_mask select from codes and may differ inside the 1e-5 tie
+ *   band of a row's threshold).
  * - Every GPU that loads the library holds the 64 MiB until the process exits.
  * - Every call looks up the array's device address on the calling thread's
  *   current device (cudaGetSymbolAddress; nothing is cached, so a context

@@ -118,3 +118,21 @@ def attention_errors(op: torch.Tensor, qp_bits, kp_bits, vp_bits, gpu_dense, ite
     if lerrs:
         out["lse_max_abs"] = float(np.concatenate(lerrs).max())
     return out
+
+
+def full_size_items(BH, Tb, sink_first, n_random=64, seed=1):
+    """Query blocks compared at full size: every sink row of the first and the
+    last head (the longest rows: every key block, the most rescales), 64
+    random non-sink blocks in each of four heads spread over the heads, and
+    the ragged last block of the first and last head."""
+    rng = np.random.default_rng(seed)
+    heads = sorted({0, BH // 3, (2 * BH) // 3, BH - 1})
+    upper = sink_first if 0 <= sink_first < Tb else Tb
+    items = []
+    if 0 <= sink_first < Tb:
+        items += [(h, i) for h in (0, BH - 1) for i in range(sink_first, Tb)]
+    for h in heads:
+        picks = rng.choice(upper, size=min(n_random, upper), replace=False)
+        items += [(h, int(i)) for i in picks]
+    items += [(0, Tb - 1), (BH - 1, Tb - 1)]
+    return sorted(set(items))

@@ -58,9 +58,15 @@ def test_query_matches_oracle_readings(L, name):
     assert sz.num_rows == BH * Tb
     s0 = Tb if sz.sink_first < 0 else sz.sink_first
     assert sz.col_idx_capacity == BH * (s0 * sz.row_capacity + (Tb - s0) * Tb)
-    means = (2 * BH * Tb * wl.head_dim * 4 + 255) // 256 * 256
+    r256 = lambda b: (b + 255) // 256 * 256
+    means = r256(2 * BH * Tb * wl.head_dim * 4)
     scores_per_head = Tb * ((Tb + 3) // 4 * 4) * 4
-    assert sz.mask_workspace_bytes == 2 * means + min(BH, max(1, (96 << 20) // scores_per_head)) * scores_per_head
+    score_group = min(BH, max(1, (96 << 20) // scores_per_head)) * scores_per_head
+    items = BH * ((Tb + 127) // 128)          # (head, 128 query blocks)
+    # coarse and fine code bytes, histograms, code widths, overflow list
+    codes = (2 * r256(items * ((Tb + 31) // 32) * 128 * 8 * 4) + r256(items * 2 * 16 * 128 * 4)
+             + r256(items * 128 * 4) + r256(4 * (BH * Tb + 1)))
+    assert sz.mask_workspace_bytes == 2 * means + max(score_group, codes)
 
 
 def test_keep_ratio_matches_oracle(L):

@@ -18,7 +18,8 @@ import oracle
 from image_dits_b200 import build as rf2_build
 from image_dits_b200 import rf2
 from image_dits_b200.workload import WORKLOADS, Workload, make_qkv
-from parity import (ATTN_MAX_ABS, ATTN_MEAN_ABS, attention_errors, bits, check_csr, compare_masks, run_path)
+from parity import (ATTN_MAX_ABS, ATTN_MEAN_ABS, attention_errors, bits, check_csr, compare_masks,
+                    full_size_items, run_path)
 
 pytestmark = pytest.mark.gpu
 
@@ -99,15 +100,17 @@ def test_image_parity(name):
 
 @pytest.mark.parametrize("d,T,H,W", [(128, 3, 16, 24), (64, 2, 20, 21), (128, 1, 64, 64)])
 def test_pooled_scores_precision(d, T, H, W):
-    """The tensor-core pooled scores (tf32 hi/lo products) left in the mask
-    workspace agree with the fp64 oracle's S^ to well inside the 1e-5 band."""
+    """The tensor-core pooled scores (tf32 hi/lo products) agree with the fp64
+    oracle's S^ to well inside the 1e-5 band.  The CDF-threshold path leaves
+    them in the mask workspace (the top-n path never writes them out; it
+    uses the same three products)."""
     rope = (0, d // 2, d // 2) if T == 1 else ((24, 20, 20) if d == 64 else (44, 42, 42))
     wl = Workload("scores", 1, 3, d, T, H, W, 1, 8, 8, 0.3, T > 1, rope)
     q, k, _ = make_qkv(wl, "cuda", seed=17)
     g = rf2.geometry_of(wl)
     qp, kp = rf2.permute(g, q), rf2.permute(g, k)
-    mask, ws = rf2.alloc_mask(g, wl.keep, qp.device)
-    rf2.predict_mask(g, qp, kp, wl.keep, mask, ws)
+    mask, ws = rf2.alloc_mask(g, 1.0, qp.device)
+    rf2.predict_mask_cdf(g, qp, kp, 0.5, mask, ws)
     torch.cuda.synchronize()
     Tb = wl.num_blocks
     means_bytes = (2 * wl.heads * Tb * d * 4 + 255) // 256 * 256
@@ -257,7 +260,30 @@ def test_long_rows_selection(keep, sink):
     compare_masks(mask.dense(), bits(qp), bits(kp), keep, wl.frames, wl.height, wl.width, sink)
 
 
-def _full_size(name, n_random_blocks, n_sink_blocks):
+@pytest.mark.parametrize("name,wl", _small_cases() + [("image", WORKLOADS["image"]),
+                                                      ("long_rows", Workload("long", 1, 2, 128, 4, 64, 144, 2, 8, 8,
+                                                                             0.2, True, (44, 42, 42)))])
+def test_mask_from_codes(name, wl, monkeypatch):
+    """The selection from 16-bit score codes (the path of large calls), forced
+    on small ones: the masks match the oracle outside the tie band, and the
+    score-matrix selection on the same inputs (equal outside the band too)."""
+    q, k, v = make_qkv(wl, "cuda", seed=11)
+    g = rf2.geometry_of(wl)
+    qp, kp = rf2.permute(g, q), rf2.permute(g, k)
+    monkeypatch.setenv("RF2_MASK_SELECT", "codes")
+    mask = rf2.predict_mask(g, qp, kp, wl.keep)
+    torch.cuda.synchronize()
+    assert rf2.device_status() == rf2.RF2_OK
+    check_csr(mask, mask.sizes.sink_first)
+    dense = mask.dense()
+    compare_masks(dense, bits(qp), bits(kp), wl.keep, wl.frames, wl.height, wl.width, wl.sink, wl.text_tokens)
+    monkeypatch.setenv("RF2_MASK_SELECT", "scores")
+    ref = rf2.predict_mask(g, qp, kp, wl.keep).dense()
+    differ = int((dense != ref).sum())
+    assert differ <= max(4, 1e-4 * dense.size), differ
+
+
+def _full_size(name):
     wl = WORKLOADS[name]
     q, k, v = make_qkv(wl, "cuda", seed=0)
     g = rf2.geometry_of(wl)
@@ -275,27 +301,26 @@ def _full_size(name, n_random_blocks, n_sink_blocks):
     # these inputs they are a fraction of a percent (pooled scores cluster).
     print(f"{name}: mask compared exactly on {compared} blocks, {excluded} in the 1e-5 tie band")
     assert excluded <= 1e-2 * compared
-    rng = np.random.default_rng(1)
     Tb = sz.num_blocks
-    BH = wl.heads
-    items = [(int(rng.integers(0, BH)), int(rng.integers(0, sz.sink_first))) for _ in range(n_random_blocks)]
-    items += [(int(rng.integers(0, BH)), int(rng.integers(sz.sink_first, Tb))) for _ in range(n_sink_blocks)]
-    items += [(BH - 1, Tb - 1), (0, Tb - 1)]             # ragged last block
+    items = full_size_items(wl.heads, Tb, sz.sink_first)
+    n_sink = sum(1 for _, i in items if sz.sink_first >= 0 and i >= sz.sink_first)
     e = attention_errors(out["op"], qp_b, kp_b, vp_b, dense, items=items)
+    print(f"{name}: attention compared on {len(items)} query blocks ({n_sink} sink rows), "
+          f"{e['n']} values: max-abs {e['max_abs']:.3g}, mean-abs {e['mean_abs']:.3g}")
     assert e["max_abs"] <= ATTN_MAX_ABS and e["mean_abs"] <= ATTN_MEAN_ABS, e
     assert np.array_equal(bits(out["o"][:, :2]), oracle.unpermute(bits(out["op"][:, :2]), perm))
 
 
 def test_video480p_full_size():
-    _full_size("video480p", 48, 4)
+    _full_size("video480p")
 
 
 def test_video480p_text_full_size():
-    _full_size("video480p_text", 32, 4)
+    _full_size("video480p_text")
 
 
 def test_video720p_full_size():
-    _full_size("video720p", 48, 4)
+    _full_size("video720p")
 
 
 def test_device_status_clean():

@@ -6,9 +6,11 @@ cudaMalloc's implicit synchronization is not acceptable).  For them the
 library keeps a fixed 64 MiB scratch array of its own.  These tests call the
 variant through the C ABI and check that, on two calls in a row with
 different problems, its block mask is identical to the one rf2_predict_mask
-writes with a caller-supplied workspace (masks are compared exactly, as the
-other parity tests compare them), and that a problem needing more scratch
-than the array holds is refused before anything is launched.
+writes with a caller-supplied workspace and the same selection (the static
+variant always selects from the score matrix, so the reference call is made
+with RF2_MASK_SELECT=scores; masks are compared exactly), and that a problem
+needing more scratch than the array holds is refused before anything is
+launched.
 
 Kept in a file of its own that pytest collects last.
 """
@@ -42,6 +44,11 @@ def _same(a: rf2.BlockMask, b: rf2.BlockMask):
     assert torch.equal(a.row_count, b.row_count)
     ra, rb = a.dense(), b.dense()
     assert (ra == rb).all()
+
+
+@pytest.fixture(autouse=True)
+def _score_matrix_selection(monkeypatch):
+    monkeypatch.setenv("RF2_MASK_SELECT", "scores")
 
 
 def test_static_scratch_matches_workspace_variant():
