@@ -31,15 +31,21 @@
 // S buffers; P (bf16) is written over the first 32 columns of its S buffer
 // and read by the PV product straight from TMEM.  Issue order of the MMA
 // thread: S_0, S_1, then per entry e: PV_e, S_{e+2} (S_{e+2} overwrites the
-// buffer PV_e reads; the tensor pipe runs one thread's MMAs in order).
+// buffer PV_e reads; the tensor pipe runs one thread's MMAs in order).  One
+// completion barrier per product, as every tcgen05.commit (and every branch)
+// between a thread's MMAs costs the issuing thread about 50 cycles: s_full[b]
+// (S_e done: scores ready, K stage b free) and pv_done[b] (PV_e done: V stage
+// b free, O holds entry e).
 //
 // Softmax (eqs. (2)-(4)) in fp32, log2 domain, per thread and entry: the 64
-// scores are loaded once, their max taken, then P written in bf16 and the
-// row sum accumulated.  The running max m is raised (and O rescaled in TMEM)
-// only when an entry's max exceeds it by more than 8 (a factor 256); O and l
-// always use the same m, so O / l is unchanged.  Before a rescale the warp
-// waits for PV_{e-1} (barrier o_done, one phase per PV): S_e completing
-// implies PV_{e-2} has, but PV_{e-1} may still run.
+// scores are loaded once and P = 2^(s - m) is written in bf16 under the
+// running max m as it stands, the row sum accumulated.  No max is taken
+// unless the row has none yet or the entry's sum exceeds 2^24 (P stays a
+// valid bf16 and O, l far inside fp32 below that); then m is raised to the
+// entry's max, O rescaled in TMEM and P written again.  O and l always use
+// the same m, so O / l is unchanged.  Before a rescale the warp
+// waits for PV_{e-1} (barrier pv_done): S_e completing implies PV_{e-2}
+// has, but PV_{e-1} may still run.
 //
 // Every wait on an mbarrier is bounded (ptx.cuh): on a timeout the CTA
 // raises a shared abort flag, every role leaves its loop, in-flight TMA loads
@@ -78,10 +84,9 @@ struct AttnCfg {
 
 struct __align__(16) AttnCtl {
     uint64_t q_full;
-    uint64_t k_full[2], k_empty[2];
-    uint64_t v_full[2], v_empty[2];
-    uint64_t s_full[2], p_full[2];
-    uint64_t o_done, o_final, drain;
+    uint64_t k_full[2], v_full[2];
+    uint64_t s_full[2], p_full[2], pv_done[2];
+    uint64_t o_final, drain;
     uint32_t tmem_base;
     int32_t list_len;
     int32_t abort;
@@ -101,6 +106,10 @@ struct AttnArgs {
     int32_t sink_pairs;     // pairs holding a sink block (the last ones of a head): scheduled early
     float scale_log2;       // log2(e) / sqrt(D)
 };
+
+// An entry's probability sum under a stale running max up to which its P is
+// used as it is (P <= 2^24 in bf16, and O, l stay far inside fp32).
+constexpr float kSumLimit = 16777216.f;
 
 // 32 scores of one row -> 16 packed bf16 pairs of P = 2^(s*sl2 - m), adding
 // the fp32 probabilities to sum4; x = s*sl2 - m and the sums run two lanes
@@ -193,13 +202,11 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         #pragma unroll
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&ctl->k_full[b]), 1);
-            mbar_init(smem_u32(&ctl->k_empty[b]), 1);
             mbar_init(smem_u32(&ctl->v_full[b]), 1);
-            mbar_init(smem_u32(&ctl->v_empty[b]), 1);
             mbar_init(smem_u32(&ctl->s_full[b]), 1);
             mbar_init(smem_u32(&ctl->p_full[b]), 128);
+            mbar_init(smem_u32(&ctl->pv_done[b]), 1);
         }
-        mbar_init(smem_u32(&ctl->o_done), 1);
         mbar_init(smem_u32(&ctl->o_final), 1);
         mbar_init(smem_u32(&ctl->drain), 1);
         ctl->abort = 0;
@@ -299,7 +306,8 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint32_t dst = base_u32 + Cfg::OFF_K + g * Cfg::KV_BLOCK;
             int issued = -1;
             for (int e = g, i = 0; e < L; e += 2, ++i) {
-                if (i > 0 && !mbar_wait(smem_u32(&ctl->k_empty[g]), (i - 1) & 1, abort, args.status)) break;
+                // stage g is free once S_{e-2} is done
+                if (i > 0 && !mbar_wait(smem_u32(&ctl->s_full[g]), (i - 1) & 1, abort, args.status)) break;
                 const int j = block_of(e);
                 mbar_arrive_expect_tx(full, Cfg::KV_BLOCK);
                 for (int c = 0; c < Cfg::KCH; ++c)
@@ -317,7 +325,8 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             int issued = -1;                     // entries e <= issued were loaded
             for (int e = 0; e < L; ++e) {
                 const int b = e & 1, i = e >> 1;
-                if (i > 0 && !mbar_wait(smem_u32(&ctl->v_empty[b]), (i - 1) & 1, abort, args.status)) break;
+                // stage b is free once PV_{e-2} is done
+                if (i > 0 && !mbar_wait(smem_u32(&ctl->pv_done[b]), (i - 1) & 1, abort, args.status)) break;
                 mbar_arrive_expect_tx(smem_u32(&ctl->v_full[b]), Cfg::KV_BLOCK);
                 tma_load_4d(base_u32 + Cfg::OFF_V + b * Cfg::KV_BLOCK, &tm_v, smem_u32(&ctl->v_full[b]), 0,
                             block_of(e) * 64, 0, (int)bh);
@@ -332,24 +341,24 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0);
             constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 1);
-            const uint32_t q_s = base_u32 + Cfg::OFF_Q;
-            const uint32_t k_s = base_u32 + Cfg::OFF_K;
-            const uint32_t v_s = base_u32 + Cfg::OFF_V;
+            // descriptors: only the start address (16-byte units, low 14 bits) changes
+            const uint64_t dq = smem_desc_sw128(base_u32 + Cfg::OFF_Q, 16, 1024);
+            const uint64_t dk = smem_desc_sw128(base_u32 + Cfg::OFF_K, 16, 1024);
+            const uint64_t dv = smem_desc_sw128(base_u32 + Cfg::OFF_V, 64 * 128, 1024);
             // S_e = Q K_e^T into S buffer e mod 2
             auto issue_s = [&](int e) -> bool {
                 const int b = e & 1;
                 if (!mbar_wait(smem_u32(&ctl->k_full[b]), (e >> 1) & 1, abort, args.status)) return false;
                 tc_fence_after();
-                const uint32_t kb = k_s + b * Cfg::KV_BLOCK;
+                const uint64_t kb = dk + ((b * Cfg::KV_BLOCK) >> 4);
                 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk & 3) * 32;          // 16 bf16 = 32 bytes per K step
-                    const uint64_t a = smem_desc_sw128(q_s + (kk >> 2) * Cfg::Q_CHUNK + off, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * Cfg::KB_CHUNK + off, 16, 1024);
-                    mma_ss(tmem + Cfg::TM_S + 64 * b, a, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                    // 16 bf16 = 32 bytes per K step
+                    const uint32_t off = ((kk >> 2) * Cfg::Q_CHUNK + (kk & 3) * 32) >> 4;
+                    const uint32_t offk = ((kk >> 2) * Cfg::KB_CHUNK + (kk & 3) * 32) >> 4;
+                    mma_ss(tmem + Cfg::TM_S + 64 * b, dq + off, kb + offk, IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(smem_u32(&ctl->s_full[b]));
-                mma_commit(smem_u32(&ctl->k_empty[b]));
                 return true;
             };
             bool ok = (L == 0) || mbar_wait(smem_u32(&ctl->q_full), 0, abort, args.status);
@@ -361,16 +370,14 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (!mbar_wait(smem_u32(&ctl->p_full[b]), par, abort, args.status)) break;
                 if (!mbar_wait(smem_u32(&ctl->v_full[b]), par, abort, args.status)) break;
                 tc_fence_after();
-                const uint32_t vb = v_s + b * Cfg::KV_BLOCK;
+                const uint64_t vb = dv + ((b * Cfg::KV_BLOCK) >> 4);
                 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     // 16 keys per K step; V as the MN-major B operand (d chunks 8 KB apart)
-                    const uint64_t bd = smem_desc_sw128(vb + kk * 2048, 64 * 128, 1024);
-                    mma_ts(tmem + Cfg::TM_O, tmem + Cfg::TM_S + 64 * b + kk * 8, bd, IDESC_O,
+                    mma_ts(tmem + Cfg::TM_O, tmem + Cfg::TM_S + 64 * b + kk * 8, vb + ((kk * 2048) >> 4), IDESC_O,
                            (e > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(smem_u32(&ctl->v_empty[b]));
-                mma_commit(smem_u32(&ctl->o_done));
+                mma_commit(smem_u32(&ctl->pv_done[b]));
                 if (e == L - 1) mma_commit(smem_u32(&ctl->o_final));
                 if (e + 2 < L) ok = issue_s(e + 2);
             }
@@ -406,39 +413,58 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tmem_wait_ld();
                 reg_fence(a);
                 reg_fence(c);
-                float mx;
-                if (nv == 64) mx = max_chunk<false>(c, 32, max_chunk<false>(a, 32, -INFINITY));
-                else mx = max_chunk<true>(c, nv - 32, max_chunk<true>(a, nv, -INFINITY));
-                const float mb = mx * sl2;                 // scale > 0: max commutes
-                const bool need = (m_run != -INFINITY) && (mb > m_run + 8.0f);
-                if (__any_sync(0xffffffffu, need)) {
-                    // Rescale O once PV_{e-1} has completed (S_e done implies PV_{e-2} is).
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait(smem_u32(&ctl->o_done), (uint32_t)((e - 1) & 1), abort, args.status));
-                    if (!ok) break;
-                    tc_fence_after();
-                    float f = 1.f;
-                    if (need) { f = ex2_approx(m_run - mb); l_run *= f; m_run = mb; }
-                    #pragma unroll 1
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_addr + Cfg::TM_O + c0, o);
-                        tmem_wait_ld();
-                        reg_fence(o);
-                        #pragma unroll
-                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
-                        tmem_st32(tmem + lane_addr + Cfg::TM_O + c0, o);
-                    }
-                }
-                if (m_run == -INFINITY) m_run = mb;
-                const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
                 // P = 2^(s*sl2 - m) in bf16 over the first 32 columns of the buffer
-                if (nv == 64) exp_chunk<false>(a, sl2, neg_mu, 32, pk, sum4);
-                else exp_chunk<true>(a, sl2, neg_mu, nv, pk, sum4);
-                tmem_st16(s_row, pk);
-                if (nv == 64) exp_chunk<false>(c, sl2, neg_mu, 32, pk, sum4);
-                else exp_chunk<true>(c, sl2, neg_mu, nv - 32, pk, sum4);
-                tmem_st16(s_row + 16, pk);
+                auto exps = [&](float neg_mu) {
+                    #pragma unroll
+                    for (int k = 0; k < 4; ++k) sum4[k] = 0.f;
+                    if (nv == 64) exp_chunk<false>(a, sl2, neg_mu, 32, pk, sum4);
+                    else exp_chunk<true>(a, sl2, neg_mu, nv, pk, sum4);
+                    tmem_st16(s_row, pk);
+                    if (nv == 64) exp_chunk<false>(c, sl2, neg_mu, 32, pk, sum4);
+                    else exp_chunk<true>(c, sl2, neg_mu, nv - 32, pk, sum4);
+                    tmem_st16(s_row + 16, pk);
+                };
+                // Fast path: the entry's probabilities under the running max as it
+                // stands, with no max taken; it holds while their sum stays within
+                // kSumLimit.  A row's first kept entry, or a sum above the limit
+                // (or not finite), takes the entry's max instead, raises m (O
+                // rescaled) and writes P again before the hand-off.
+                bool slow = (m_run == -INFINITY);
+                if (!slow) {
+                    exps(-m_run);
+                    slow = !((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]) <= kSumLimit);
+                }
+                if (__any_sync(0xffffffffu, slow)) {
+                    float mb = m_run;
+                    if (slow) {
+                        float mx;
+                        if (nv == 64) mx = max_chunk<false>(c, 32, max_chunk<false>(a, 32, -INFINITY));
+                        else mx = max_chunk<true>(c, nv - 32, max_chunk<true>(a, nv, -INFINITY));
+                        mb = mx * sl2;                     // scale > 0: max commutes
+                    }
+                    const bool resc = slow && (m_run != -INFINITY) && (mb > m_run);
+                    if (__any_sync(0xffffffffu, resc)) {
+                        // Rescale O once PV_{e-1} has completed (S_e done implies PV_{e-2} is).
+                        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl->pv_done[(e - 1) & 1]),
+                                                               (uint32_t)(((e - 1) >> 1) & 1), abort, args.status));
+                        if (!ok) break;
+                        tc_fence_after();
+                        float f = 1.f;
+                        if (resc) { f = ex2_approx(m_run - mb); l_run *= f; }
+                        #pragma unroll 1
+                        for (int c0 = 0; c0 < D; c0 += 32) {
+                            uint32_t o[32];
+                            tmem_ld32(tmem + lane_addr + Cfg::TM_O + c0, o);
+                            tmem_wait_ld();
+                            reg_fence(o);
+                            #pragma unroll
+                            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+                            tmem_st32(tmem + lane_addr + Cfg::TM_O + c0, o);
+                        }
+                    }
+                    if (slow && (m_run == -INFINITY || mb > m_run)) m_run = mb;
+                    exps(m_run == -INFINITY ? 0.f : -m_run);
+                }
             } else {
                 #pragma unroll
                 for (int k = 0; k < 16; ++k) pk[k] = 0u;

@@ -144,14 +144,17 @@ def test_constant_value_rows():
     assert err <= 2 ** -7 * v.float().abs().max().item() + 1e-6
 
 
-@pytest.mark.parametrize("d,keep", [(128, 1.0), (128, 0.5), (64, 0.4)])
-def test_running_max_rescale(d, keep):
-    """Key blocks in four groups whose scores step up by about 9 (log2 units)
-    from one group to the next, and query rows alternating in sign: rows whose
-    scores rise raise their running max, and O is rescaled, at the group
-    boundaries, while the other rows of the same warp keep their first max;
-    under a sparse mask (chosen on the unmodified scores) the steps fall at
-    different entries for the two query blocks of a tile."""
+@pytest.mark.parametrize("d,keep,step", [(128, 1.0, 30.0), (128, 0.5, 30.0), (64, 0.4, 30.0), (128, 0.5, 9.0)])
+def test_running_max_rescale(d, keep, step):
+    """Key blocks in four groups whose scores step up by `step` (log2 units)
+    from one group to the next, and query rows alternating in sign.  With
+    steps of 30 an entry's probabilities under the old running max sum past
+    2^24 at a group boundary: those rows take the entry's max, raise their
+    running max and rescale O, while the other rows of the same warp keep
+    their first max; with steps of 9 the probabilities are used under the
+    stale max (up to 2^9 each).  Under a sparse mask (chosen on the
+    unmodified scores) the steps fall at different entries for the two query
+    blocks of a tile."""
     rope = (44, 42, 42) if d == 128 else (24, 20, 20)
     wl = Workload("rescale", 1, 2, d, 4, 16, 16, 2, 4, 4, keep, False, rope)
     g = rf2.geometry_of(wl)
@@ -164,7 +167,7 @@ def test_running_max_rescale(d, keep):
     sign = torch.where(torch.arange(N, device="cuda") % 2 == 0, 1.0, -1.0)
     qp[..., 0] = (A * sign).to(qp.dtype)
     group = (torch.arange(N, device="cuda") // 64) * 4 // Tb
-    kp[..., 0] = (9.0 * group / (sl2 * A)).to(kp.dtype)
+    kp[..., 0] = (step * group / (sl2 * A)).to(kp.dtype)
     lse = torch.full((wl.heads * N,), float("nan"), device="cuda")
     op = rf2.block_sparse_attn(g, qp, kp, vp, mask, lse=lse)
     torch.cuda.synchronize()
