@@ -769,10 +769,11 @@ __global__ void __launch_bounds__(256) topn_overflow_kernel(const TopnArgs args)
 //      64 keys in bin b*, more than 16 keys of c* to rank, more than 4 keys
 //      tied in the fine code, or its threshold in a saturated code (0 or 255:
 //      the bracket missed) is listed for topn_overflow_kernel.
-//   4. The warp writes its rows one by one: each lane expands the kept bits of
-//      two bitmap words into shared memory at its offset (a warp scan of the
-//      words' counts), and the row leaves in full-line stores, the sink columns
-//      last; sink rows (and keep = 1) keep every block.
+//   4. Each half-warp writes one row at a time: each lane expands the kept bits
+//      of four bitmap words into shared memory at its offset (a scan of the
+//      words' counts over the half-warp), and the row leaves in 64-byte
+//      stores, the sink columns last; sink rows (and keep = 1) keep every
+//      block.
 template <int D>
 __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
 {
@@ -789,9 +790,10 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
     const int row_end = min(mg.sink_first, Tb);
     const int sf = mg.sink_first;                          // <= Tb
     uint32_t* bm = reinterpret_cast<uint32_t*>(smem_raw);              // [32][BS]
+    const int SH = max(BCAP * 32, 2 * n) / 2;              // staging entries per half-warp (>= n)
     uint32_t* cand = bm + 32 * BS;                                       // [BCAP][32]: code16 << 16 | j
-    int32_t* stage = reinterpret_cast<int32_t*>(cand);                   // then: the row being written (<= 2048)
-    int32_t* kind = reinterpret_cast<int32_t*>(cand + BCAP * 32);        // [32]: row kind
+    int32_t* stage = reinterpret_cast<int32_t*>(cand);                   // then: [2][SH] rows being written
+    int32_t* kind = reinterpret_cast<int32_t*>(cand + 2 * SH);           // [32]: row kind
     const int64_t units = args.BH * mtiles * 4;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
         const int64_t item = u >> 2;
@@ -825,18 +827,28 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
             const size_t wbase = (size_t)item * W8 * 128 + rl;
             const uint32_t* cw = args.codes + wbase;
             const uint32_t* fw = args.fine + wbase;
+            const float width = args.width[item * 128 + rl];       // loaded early: used after the pass
             int nb = 0;
-            uint32_t nxt[8];
+            // codes and fine bytes of groups g + 1 and g + 2 in flight while group g is read
+            uint32_t ca[8], fa[8], cb[8], fb[8];
             #pragma unroll
-            for (int k = 0; k < 8; ++k) nxt[k] = cw[(size_t)k * 128];
+            for (int k = 0; k < 8; ++k) {
+                ca[k] = cw[(size_t)k * 128];
+                fa[k] = fw[(size_t)k * 128];
+                cb[k] = (G > 1) ? cw[(size_t)(8 + k) * 128] : 0u;
+                fb[k] = (G > 1) ? fw[(size_t)(8 + k) * 128] : 0u;
+            }
             #pragma unroll 1
             for (int g = 0; g < G; ++g) {
-                uint32_t w[8];
+                uint32_t w[8], f[8];
                 #pragma unroll
-                for (int k = 0; k < 8; ++k) w[k] = nxt[k];
-                if (g + 1 < G) {
+                for (int k = 0; k < 8; ++k) { w[k] = ca[k]; f[k] = fa[k]; ca[k] = cb[k]; fa[k] = fb[k]; }
+                if (g + 2 < G) {
                     #pragma unroll
-                    for (int k = 0; k < 8; ++k) nxt[k] = cw[(size_t)(8 * (g + 1) + k) * 128];
+                    for (int k = 0; k < 8; ++k) {
+                        cb[k] = cw[(size_t)(8 * (g + 2) + k) * 128];
+                        fb[k] = fw[(size_t)(8 * (g + 2) + k) * 128];
+                    }
                 }
                 const int nv = Tb - 32 * g;
                 const uint32_t vm = (nv >= 32) ? 0xffffffffu : ((1u << nv) - 1u);
@@ -847,19 +859,14 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
                     inb |= bytes_eq(w[k] & 0xF8F8F8F8u, pat_bin) << (4 * k);
                 }
                 inb &= vm;
-                if (inb) {
-                    uint32_t f[8];
-                    #pragma unroll
-                    for (int k = 0; k < 8; ++k) f[k] = fw[(size_t)(8 * g + k) * 128];
-                    do {
-                        const int b = __ffs(inb) - 1;
-                        inb &= inb - 1;
-                        if (nb < BCAP) {
-                            const uint32_t code16 = (byte_of8(w, b) << 8) | byte_of8(f, b);
-                            cand[nb * 32 + lane] = (code16 << 16) | (uint32_t)(32 * g + b);
-                        }
-                        ++nb;
-                    } while (inb);
+                while (inb) {
+                    const int b = __ffs(inb) - 1;
+                    inb &= inb - 1;
+                    if (nb < BCAP) {
+                        const uint32_t code16 = (byte_of8(w, b) << 8) | byte_of8(f, b);
+                        cand[nb * 32 + lane] = (code16 << 16) | (uint32_t)(32 * g + b);
+                    }
+                    ++nb;
                 }
                 brow[g] = bits & vm;
             }
@@ -885,7 +892,6 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
                 }
                 const uint32_t cstar = (uint32_t)(bstar * 8 + sub);
                 const bool partial = need < m;
-                const float width = args.width[item * 128 + rl];
                 const bool tiny = cstar > 0 && cstar < 255 && width <= args.tiny_width;
                 const bool ranked = partial && !tiny;
                 uint32_t kept_mask = 0;                        // bit e: the e-th key of c* (j order) is kept
@@ -1015,47 +1021,59 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
         }
         kind[lane] = rk;
         __syncwarp();
-        // 4. the CSR rows of the warp's 32 query blocks
+        // 4. the CSR rows of the warp's 32 query blocks, two at a time: half-warp h
+        // writes rows 16 h + r; lane l of it holds bitmap words 4 l .. 4 l + 3
         const int wl = (sf + 31) >> 5;                     // bitmap words below the sink columns
+        const int hw = lane >> 4, hl = lane & 15;
+        const unsigned hmask = 0xFFFFu << (16 * hw);
+        int32_t* hstage = stage + hw * SH;
         #pragma unroll 1
-        for (int rr = 0; rr < 32; ++rr) {
+        for (int r0 = 0; r0 < 16; ++r0) {
+            const int rr = 16 * hw + r0;
             const int k = kind[rr];
-            if (k >= 2) continue;                              // no row, or the warp kernel writes it
+            if (k >= 2) continue;                              // no row, or the overflow kernel writes it
             const int ir = m0 + (rl - lane) + rr;
             const int64_t row_id = bh * Tb + ir;
             const int64_t rs = row_offset(mg, bh, ir);
             int32_t* out = args.col_idx + rs;
             if (k == 1) {
-                for (int j = lane; j < Tb; j += 32) out[j] = j;
-                if (lane == 0) { args.row_start[row_id] = (int32_t)rs; args.row_count[row_id] = Tb; }
+                for (int j = hl; j < Tb; j += 16) out[j] = j;
+                if (hl == 0) { args.row_start[row_id] = (int32_t)rs; args.row_count[row_id] = Tb; }
                 continue;
             }
             const uint32_t* brow = bm + rr * BS;
-            auto below = [&](int wi) -> uint32_t {
-                if (wi >= wl) return 0u;
-                const uint32_t x = brow[wi];
-                const int j0 = 32 * wi;
-                return (j0 + 32 <= sf) ? x : (x & ((1u << (sf - j0)) - 1u));
-            };
-            uint32_t x0 = below(lane), x1 = below(lane + 32);
-            const int c0 = __popc(x0), c1 = __popc(x1);
-            int i0 = c0, i1 = c1;
+            uint32_t x[4];
+            int c = 0;
             #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int a0 = __shfl_up_sync(0xffffffffu, i0, o);
-                const int a1 = __shfl_up_sync(0xffffffffu, i1, o);
-                if (lane >= o) { i0 += a0; i1 += a1; }
+            for (int q = 0; q < 4; ++q) {
+                const int wi = 4 * hl + q;
+                uint32_t v = 0u;
+                if (wi < wl) {
+                    v = brow[wi];
+                    const int j0 = 32 * wi;
+                    if (j0 + 32 > sf) v &= (1u << (sf - j0)) - 1u;
+                }
+                x[q] = v;
+                c += __popc(v);
             }
-            const int t0 = __shfl_sync(0xffffffffu, i0, 31);
-            const int nk = t0 + __shfl_sync(0xffffffffu, i1, 31);
-            int p0 = i0 - c0, p1 = t0 + i1 - c1;               // offsets of words lane, lane + 32
-            while (x0) { const int b = __ffs(x0) - 1; x0 &= x0 - 1; stage[p0++] = 32 * lane + b; }
-            while (x1) { const int b = __ffs(x1) - 1; x1 &= x1 - 1; stage[p1++] = 32 * (lane + 32) + b; }
-            __syncwarp();
-            for (int p = lane; p < nk; p += 32) out[p] = stage[p];
-            for (int j = sf + lane; j < Tb; j += 32) out[nk + (j - sf)] = j;
-            if (lane == 0) { args.row_start[row_id] = (int32_t)rs; args.row_count[row_id] = nk + (Tb - sf); }
-            __syncwarp();
+            int incl = c;
+            #pragma unroll
+            for (int o = 1; o < 16; o <<= 1) {
+                const int a = __shfl_up_sync(hmask, incl, o, 16);
+                if (hl >= o) incl += a;
+            }
+            const int nk = __shfl_sync(hmask, incl, 15, 16);
+            int p = incl - c;
+            #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v = x[q];
+                while (v) { const int b = __ffs(v) - 1; v &= v - 1; hstage[p++] = 32 * (4 * hl + q) + b; }
+            }
+            __syncwarp(hmask);
+            for (int p2 = hl; p2 < nk; p2 += 16) out[p2] = hstage[p2];
+            for (int j = sf + hl; j < Tb; j += 16) out[nk + (j - sf)] = j;
+            if (hl == 0) { args.row_start[row_id] = (int32_t)rs; args.row_count[row_id] = nk + (Tb - sf); }
+            __syncwarp(hmask);
         }
     }
 }
