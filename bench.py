@@ -52,8 +52,8 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_desc(wl):
-    return (f"{wl.name}: B={wl.batch}/GPU, {wl.heads} heads, d={wl.head_dim}, latent {wl.frames}x{wl.height}x"
+def workload_desc(wl, per_gpu=True):
+    return (f"{wl.name}: B={wl.batch}{'/GPU' if per_gpu else ' (one call over all GPUs)'}, {wl.heads} heads, d={wl.head_dim}, latent {wl.frames}x{wl.height}x"
             f"{wl.width}{f' + {wl.text_tokens} text' if wl.text_tokens else ''} ({wl.num_tokens:,} tokens), block 64, window {wl.win_t}x{wl.win_h}x{wl.win_w}, keep "
             f"{wl.keep:g} of key blocks (sparsity {1 - wl.keep:g}) + first-frame sink={'on' if wl.sink else 'off'}")
 
@@ -75,11 +75,14 @@ def kept_flops_from_mask(mask, wl) -> float:
 
 
 # DRAM bytes (read + write) per (token, head) of one block_sparse_attn_kernel<128>
-# launch, from an ncu capture at 480p (391.2 MB / (32,760 tokens x 12 heads)).  The
-# kernel's DRAM traffic is its compulsory Q/K/V reads and O writes (K/V re-reads hit
-# L2), so it scales with the token-heads of the workload.  Re-measure whenever the
+# launch: dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture on the
+# 720p shape with 8 heads (513.53 MB + 138.92 MB over 75,600 tokens x 8 heads), of
+# the kernel as built at ATTN_TRAFFIC_BUILD.  The kernel's DRAM traffic is its
+# compulsory Q/K/V reads and O writes (1,024 B per token-head; K/V re-reads hit L2),
+# so it scales with the token-heads of the workload.  Re-measure whenever the
 # kernel changes.
-ATTN_DRAM_BYTES_PER_TOKEN_HEAD = (306.926e6 + 84.263e6) / (32760 * 12)
+ATTN_DRAM_BYTES_PER_TOKEN_HEAD = (513.530112e6 + 138.922496e6) / (75600 * 8)
+ATTN_TRAFFIC_BUILD = "e735b05"
 
 
 def mask_bytes(wl, mask) -> float:
@@ -294,6 +297,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-chunks", type=int, default=8, help="head chunks of the end-to-end pipeline")
     ap.add_argument("--sweep", action="store_true", help="also time the keep-ratio sweep (stderr)")
+    ap.add_argument("--split", default="batch", choices=["batch", "heads"],
+                    help="N > 1: one batch element per GPU (weak scaling), or one call's heads divided "
+                         "among the GPUs (strong scaling); neither exchanges data")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -326,8 +332,16 @@ def main():
         dist.barrier()
     rf2.lib()
 
+    call = wl                                       # the workload one call computes (all ranks together)
+    if args.split == "heads":
+        # one call's inputs on every rank (same seed); this rank keeps heads [h0, h1)
+        from image_dits_b200.shard import head_range
+        h0, h1 = head_range(wl.heads, world, rank)
+        q, k, v = (x[:, h0:h1].contiguous() for x in make_qkv(wl, dev, seed=rank_seed(0)))
+        wl = dataclasses.replace(wl, heads=h1 - h0)
+    else:
+        q, k, v = make_qkv(wl, dev, seed=rank_seed(rank))
     g = rf2.geometry_of(wl)
-    q, k, v = make_qkv(wl, dev, seed=rank_seed(rank))
     qp, kp, vp, op, o = (torch.empty_like(q) for _ in range(5))
     mask, ws = rf2.alloc_mask(g, 1.0 if args.tau is not None else wl.keep, dev)
     stream = torch.cuda.current_stream()
@@ -483,15 +497,17 @@ def main():
         "attn_ms_per_call": attn_ms_all,
         "attn_tflops": flops_all / world / (attn_ms_all * 1e-3) / 1e12,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if args.split == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) + 0.5*smooth 3D field, 3D RoPE on Q/K, bf16)",
-        "config": {"workload": workload_desc(wl) if args.tau is None else
-                   workload_desc(wl).split(", keep")[0] + f", CDF-threshold selection tau={args.tau:g} + first-frame "
+        "config": {"workload": workload_desc(call, args.split != "heads") if args.tau is None else
+                   workload_desc(call, args.split != "heads").split(", keep")[0] + f", CDF-threshold selection tau={args.tau:g} + first-frame "
                    f"sink={'on' if wl.sink else 'off'}",
-                   "global_batch": world * wl.batch, "seq_len": wl.num_tokens,
-                   "parallelism": f"dp{world} (independent batch element per GPU, no collective)",
+                   "global_batch": (call.batch if args.split == "heads" else world * wl.batch), "seq_len": wl.num_tokens,
+                   "parallelism": (f"heads{world} (the call's {call.heads} heads divided among {world} GPUs, "
+                                   f"{wl.heads} on rank 0; no collective)" if args.split == "heads"
+                                   else f"dp{world} (independent batch element per GPU, no collective)"),
                    "kept_pairs_per_gpu": kept_pairs, "density": density,
                    "l2": (f"inputs larger than L2 ({q.numel() * 2 / 1e6:.0f} MB per tensor), no flush" if flush is None
                           else "256 MB buffer written before every timed step; steps timed one by one")},
@@ -499,8 +515,9 @@ def main():
                      "peak": attn_peak, "unit": "TFLOP/s", "frac": attn_tf / attn_peak,
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
                      "traffic": ATTN_DRAM_BYTES_PER_TOKEN_HEAD * wl.num_tokens * wl.batch * wl.heads,
-                     "traffic_source": "dram read+write of one ncu capture at 480p, scaled by token-heads "
-                                       "(profiles/attn_video480p_ncu.md)"},
+                     "traffic_source": "dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of "
+                                       "block_sparse_attn_kernel<128> on the 720p shape with 8 heads (build "
+                                       f"{ATTN_TRAFFIC_BUILD}), scaled by token-heads"},
         "stages": stages,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
