@@ -9,6 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librf2.so")
+CHECKED_LIB = os.path.join(HERE, "librf2_checked.so")
 SOURCES = ["rf2_lib.cu"]
 DEPS = ["rf2_lib.cu", "attn.cuh", "mask.cuh", "topn.cuh", "permute.cuh", "geometry.cuh", "ptx.cuh"]
 
@@ -22,27 +23,35 @@ def nvcc_cmd(out: str, extra=()) -> list:
     ]
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, d) for d in DEPS] + [os.path.join(ROOT, "include", "rf2.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if force or _stale():
-        tmp = LIB + ".tmp"
-        r = subprocess.run(nvcc_cmd(tmp), capture_output=True, text=True)
+def _build_one(lib: str, extra, force: bool, verbose: bool):
+    if force or _stale(lib):
+        tmp = lib + ".tmp"
+        r = subprocess.run(nvcc_cmd(tmp, extra), capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
-            raise RuntimeError("nvcc failed building librf2.so")
+            raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
         if verbose:
             sys.stderr.write(r.stderr)
-        os.replace(tmp, LIB)
+        os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Builds librf2.so and its range-checked twin librf2_checked.so
+    (RF2_CHECKED=1: the same code plus index checks reported through the
+    device status word); returns the path of librf2.so."""
+    _build_one(LIB, (), force, verbose)
+    _build_one(CHECKED_LIB, ("-DRF2_CHECKED=1",), force, verbose)
     return LIB
 
 
 if __name__ == "__main__":
     build(force=True, verbose=True)
-    print(LIB)
+    print(LIB, CHECKED_LIB)

@@ -105,6 +105,7 @@ struct AttnArgs {
     int32_t pairs;          // ceil(Tb / 2)
     int32_t sink_pairs;     // pairs holding a sink block (the last ones of a head): scheduled early
     float scale_log2;       // log2(e) / sqrt(D)
+    int64_t col_capacity;   // checked build: bound of row_start + row_count (B*H*T_b^2)
 };
 
 // An entry's probability sum under a stale running max up to which its P is
@@ -235,18 +236,28 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t tmem = ctl->tmem_base;
     const int64_t rA = bh * Tb + qb0;
     {
-        const int lenA = min(max(args.row_count[rA], 0), Tb);
+        // (checked build: a row outside the CSR array, or a key block outside
+        // 0 .. T_b - 1, is reported and skipped)
+        auto row_len = [&](int64_t r) -> int {
+            const int32_t cnt = args.row_count[r];
+            const int len = min(max(cnt, 0), Tb);
+            if (RF2_CHECKED && !in_range(cnt >= 0 && cnt <= Tb && args.row_start[r] >= 0 &&
+                                         (int64_t)args.row_start[r] + cnt <= args.col_capacity))
+                return 0;
+            return len;
+        };
+        const int lenA = row_len(rA);
         const int32_t* srcA = args.col_idx + args.row_start[rA];
         for (int e = tid; e < lenA; e += Cfg::THREADS) {
             const int32_t j = srcA[e];
-            if (j >= 0 && j < Tb) atomicOr(&bmA[j >> 5], 1u << (j & 31));
+            if (in_range(j >= 0 && j < Tb) && j >= 0 && j < Tb) atomicOr(&bmA[j >> 5], 1u << (j & 31));
         }
         if (has_b) {
-            const int lenB = min(max(args.row_count[rA + 1], 0), Tb);
+            const int lenB = row_len(rA + 1);
             const int32_t* srcB = args.col_idx + args.row_start[rA + 1];
             for (int e = tid; e < lenB; e += Cfg::THREADS) {
                 const int32_t j = srcB[e];
-                if (j >= 0 && j < Tb) atomicOr(&bmB[j >> 5], 1u << (j & 31));
+                if (in_range(j >= 0 && j < Tb) && j >= 0 && j < Tb) atomicOr(&bmB[j >> 5], 1u << (j & 31));
             }
         }
     }

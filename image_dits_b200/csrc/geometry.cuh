@@ -110,6 +110,7 @@ struct MaskGeo {
     int32_t sink_first;  // first sink block, Tb when there is no sink
     int32_t cap;         // capacity of a non-sink row
     int64_t head_total;  // col_idx slots per (b, h)
+    int64_t col_capacity;  // col_idx slots in all (set by the host; checked build only)
 };
 
 // First token of the full-attention region of the permuted sequence: frame 0
@@ -130,6 +131,7 @@ RF2_HD MaskGeo make_mask_geo(int32_t N, int32_t n_keep, int32_t first_sink_token
     const int32_t n_sink = m.Tb - m.sink_first;
     m.cap = imin(m.Tb, n_keep + n_sink);
     m.head_total = (int64_t)m.sink_first * m.cap + (int64_t)n_sink * m.Tb;
+    m.col_capacity = INT64_MAX;
     return m;
 }
 

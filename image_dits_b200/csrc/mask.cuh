@@ -133,18 +133,23 @@ __global__ void __launch_bounds__(256, D == 128 ? RF2_POOL_MINB : 4) permute_poo
         #pragma unroll 1
         for (int r0 = 0; r0 < rows; r0 += kSub) {
             int32_t src = 0;
-            if (lane < kSub && r0 + lane < rows) src = perm_src(g, i * kBlock + r0 + lane);
+            if (lane < kSub && r0 + lane < rows) {
+                src = perm_src(g, i * kBlock + r0 + lane);
+                if (RF2_CHECKED && !in_range(src >= 0 && src < N)) src = -1;   // checked build: reported, skipped
+            }
             uint4 v[kLoads];
+            bool ok[kLoads];
             #pragma unroll
             for (int u = 0; u < kLoads; ++u) {
                 const int r = u * R + rsub;
                 const int32_t srow = __shfl_sync(0xffffffffu, src, r);
-                if (r0 + r < rows) v[u] = __ldcs(in + (int64_t)srow * C);
+                ok[u] = r0 + r < rows && (!RF2_CHECKED || srow >= 0);
+                if (ok[u]) v[u] = __ldcs(in + (int64_t)srow * C);
             }
             #pragma unroll
             for (int u = 0; u < kLoads; ++u) {
                 const int r = r0 + u * R + rsub;
-                if (r < rows) {
+                if (ok[u]) {
                     __stcs(out + r * C, v[u]);
                     bf16x8_accumulate(v[u], acc);
                 }
@@ -264,7 +269,7 @@ __device__ __forceinline__ void write_row(const uint32_t* rk, const MaskGeo& mg,
         const bool sel = (j < Tb) && (k > thr || (eq && eq_rank < eq_left) || j >= mg.sink_first);
         eq_left -= __popc(eq_ballot);
         const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
-        if (sel) out[written + __popc(sel_ballot & ((1u << lane) - 1u))] = j;
+        if (sel) csr_put(out, written + __popc(sel_ballot & ((1u << lane) - 1u)), j, rs, mg.col_capacity);
         written += __popc(sel_ballot);
     }
     if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = written; }
@@ -284,7 +289,7 @@ __device__ __forceinline__ void select_row(const uint32_t* rk, uint32_t* hist, c
         const int64_t rs = row_offset(mg, bh, i);
         const int64_t row_id = bh * Tb + i;
         int32_t* out = col_idx + rs;
-        for (int j = lane; j < Tb; j += 32) out[j] = j;
+        for (int j = lane; j < Tb; j += 32) csr_put(out, j, j, rs, mg.col_capacity);
         if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = Tb; }
         return;
     }
@@ -656,7 +661,7 @@ __global__ void __launch_bounds__(kSelThreads) select_probe_kernel(const float* 
     const int64_t row_id = bh * Tb + i;
     int32_t* out = col_idx + rs;
     if (i >= mg.sink_first || mg.n_keep >= Tb) {
-        for (int j = lane; j < Tb; j += 32) out[j] = j;
+        for (int j = lane; j < Tb; j += 32) csr_put(out, j, j, rs, mg.col_capacity);
         if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = Tb; }
         return;
     }
@@ -745,7 +750,7 @@ __global__ void __launch_bounds__(kSelThreads) select_probe_kernel(const float* 
         const bool sel = (j < Tb) && (k > thr || (eq && eq_rank < eq_left) || j >= mg.sink_first);
         eq_left -= __popc(eq_ballot);
         const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
-        if (sel) out[written + __popc(sel_ballot & ((1u << lane) - 1u))] = j;
+        if (sel) csr_put(out, written + __popc(sel_ballot & ((1u << lane) - 1u)), j, rs, mg.col_capacity);
         written += __popc(sel_ballot);
     }
     if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = written; }
@@ -793,7 +798,7 @@ __global__ void __launch_bounds__(32 * R) select_cdf_kernel(const float* __restr
     const int64_t row_id = bh * Tb + i;
     int32_t* out = col_idx + rs;
     if (i >= mg.sink_first) {
-        for (int j = lane; j < Tb; j += 32) out[j] = j;
+        for (int j = lane; j < Tb; j += 32) csr_put(out, j, j, rs, mg.col_capacity);
         if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = Tb; }
         return;
     }
@@ -862,7 +867,7 @@ __global__ void __launch_bounds__(32 * R) select_cdf_kernel(const float* __restr
         const bool sel = (j < Tb) && (k > thr || (eq && eq_rank < eq_left) || j >= mg.sink_first);
         eq_left -= __popc(eq_ballot);
         const uint32_t sel_ballot = __ballot_sync(0xffffffffu, sel);
-        if (sel) out[written + __popc(sel_ballot & ((1u << lane) - 1u))] = j;
+        if (sel) csr_put(out, written + __popc(sel_ballot & ((1u << lane) - 1u)), j, rs, mg.col_capacity);
         written += __popc(sel_ballot);
     }
     if (lane == 0) { row_start[row_id] = (int32_t)rs; row_count[row_id] = written; }

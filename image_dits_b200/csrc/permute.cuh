@@ -47,18 +47,21 @@ __global__ void __launch_bounds__(256, RF2_PERMUTE_MINB) permute_rows_kernel(con
             const int32_t p = (int32_t)(myrow - bh * g.N);
             const int32_t s = kForward ? perm_src(g, p) : perm_dst(g, p);
             src = bh * g.N + s;
+            if (RF2_CHECKED && !in_range(s >= 0 && s < g.N)) src = -1;     // checked build: reported, skipped
         }
         uint4 v[kLoads];
+        bool ok[kLoads];
         #pragma unroll
         for (int k = 0; k < kLoads; ++k) {
             const int r = k * R + rsub;
             const int64_t srow = __shfl_sync(0xffffffffu, src, r);
-            if (row0 + r < total_rows) v[k] = __ldcs(in + srow * C + cidx);
+            ok[k] = row0 + r < total_rows && (!RF2_CHECKED || srow >= 0);
+            if (ok[k]) v[k] = __ldcs(in + srow * C + cidx);
         }
         #pragma unroll
         for (int k = 0; k < kLoads; ++k) {
             const int r = k * R + rsub;
-            if (row0 + r < total_rows) __stcs(out + (row0 + r) * C + cidx, v[k]);
+            if (ok[k]) __stcs(out + (row0 + r) * C + cidx, v[k]);
         }
     }
 }

@@ -9,6 +9,42 @@ namespace rf2 {
 
 // Device status word bits (read back by rf2_device_status).
 constexpr int kDevErrTimeout = 1;
+constexpr int kDevErrRange = 2;          // a range check of the checked build failed
+
+// Device status word: kernels OR error bits into it; rf2_device_status
+// reads and clears it.
+__device__ int g_status_word;
+
+#ifndef RF2_CHECKED
+#define RF2_CHECKED 0
+#endif
+
+// Range check of the library built with RF2_CHECKED=1 (librf2_checked.so):
+// a false `ok` ORs kDevErrRange into the device status word and the caller
+// skips the access.  In the normal build the checks are not compiled.
+__device__ __forceinline__ bool in_range(bool ok)
+{
+#if RF2_CHECKED
+    if (!ok) atomicOr(&g_status_word, kDevErrRange);
+    return ok;
+#else
+    (void)ok;
+    return true;
+#endif
+}
+
+// col_idx store of a CSR writer: out = col_idx + rs; the checked build also
+// checks rs + k against the array's capacity.
+__device__ __forceinline__ void csr_put(int32_t* out, int64_t k, int32_t v, int64_t rs, int64_t capacity)
+{
+#if RF2_CHECKED
+    if (!in_range(rs + k >= 0 && rs + k < capacity)) return;
+#else
+    (void)rs;
+    (void)capacity;
+#endif
+    out[k] = v;
+}
 
 // A bounded wait gives up after this long (ns of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

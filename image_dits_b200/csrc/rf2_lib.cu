@@ -22,10 +22,6 @@
 
 namespace rf2 {
 
-// Device status word: kernels OR error bits into it; rf2_device_status
-// reads and clears it.
-__device__ int g_status_word;
-
 // Top-n selection keeps rows of up to this many key blocks in registers
 // (select_probe_kernel, 16 keys per lane); see launch_select_topn.
 constexpr int32_t kSelectRegMaxBlocks = 32 * 16;
@@ -125,6 +121,7 @@ static int sizes_for(const rf2_geometry* g, double keep, Checked& c, MaskGeo& mg
     if (st != RF2_OK) return st;
     mg = make_mask_geo(c.N, n, sink_first_token(c.pg, g->first_frame_sink));
     const int64_t total = c.BH * mg.head_total;
+    mg.col_capacity = total;
     if (total > INT32_MAX) return RF2_ERR_UNSUPPORTED;
     if (out) {
         out->num_tokens = c.N;
@@ -329,6 +326,7 @@ static int launch_attn(const Checked& c, const MaskGeo& mg, const void* qp, cons
     a.pairs = (c.Tb + 1) / 2;
     a.sink_pairs = (mg.sink_first < c.Tb) ? a.pairs - mg.sink_first / 2 : 0;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    a.col_capacity = c.BH * (int64_t)c.Tb * c.Tb;      // the largest layout the library writes
     const size_t smem = Cfg::smem_bytes(c.Tb);
     if (ensure_dynamic_smem(reinterpret_cast<const void*>(block_sparse_attn_kernel<D>), smem) != RF2_OK)
         return RF2_ERR_CUDA;
@@ -627,6 +625,7 @@ const char* rf2_status_string(int status)
     case RF2_ERR_INSUFFICIENT_WORKSPACE: return "workspace too small";
     case RF2_ERR_CUDA: return "CUDA error";
     case RF2_ERR_TIMEOUT: return "device wait timed out";
+    case RF2_ERR_RANGE: return "index out of range (checked build)";
     default: return "unknown status";
     }
 }
@@ -865,6 +864,7 @@ int rf2_device_status(void* stream)
     if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof v) != cudaSuccess) return RF2_ERR_CUDA;
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero) != cudaSuccess) return RF2_ERR_CUDA;
+    if (v & kDevErrRange) return RF2_ERR_RANGE;
     return (v & kDevErrTimeout) ? RF2_ERR_TIMEOUT : RF2_OK;
 }
 

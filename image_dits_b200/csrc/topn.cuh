@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(256) topn_overflow_kernel(const TopnArgs args)
         int32_t* out = args.col_idx + rs;
         if (i >= row_end || n >= Tb) {                     // not listed by topn_rows_kernel; kept for safety
             if (warp == 0) {
-                for (int j = lane; j < Tb; j += 32) out[j] = j;
+                for (int j = lane; j < Tb; j += 32) csr_put(out, j, j, rs, mg.col_capacity);
                 if (lane == 0) { args.row_start[row] = (int32_t)rs; args.row_count[row] = Tb; }
             }
             continue;
@@ -742,9 +742,9 @@ __global__ void __launch_bounds__(256) topn_overflow_kernel(const TopnArgs args)
             }
             const int total = __shfl_sync(0xffffffffu, at, 31);
             at -= c;
-            while (keep) { const int b = __ffs(keep) - 1; keep &= keep - 1; out[at++] = 4 * w0 + b; }
-            while (keep2) { const int b = __ffs(keep2) - 1; keep2 &= keep2 - 1; out[at++] = 4 * w0 + 32 + b; }
-            for (int j = sf + lane; j < Tb; j += 32) out[total + (j - sf)] = j;
+            while (keep) { const int b = __ffs(keep) - 1; keep &= keep - 1; csr_put(out, at++, 4 * w0 + b, rs, mg.col_capacity); }
+            while (keep2) { const int b = __ffs(keep2) - 1; keep2 &= keep2 - 1; csr_put(out, at++, 4 * w0 + 32 + b, rs, mg.col_capacity); }
+            for (int j = sf + lane; j < Tb; j += 32) csr_put(out, total + (j - sf), j, rs, mg.col_capacity);
             if (lane == 0) { args.row_start[row] = (int32_t)rs; args.row_count[row] = total + (Tb - sf); }
         }
         __syncthreads();
@@ -1037,7 +1037,7 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
             const int64_t rs = row_offset(mg, bh, ir);
             int32_t* out = args.col_idx + rs;
             if (k == 1) {
-                for (int j = hl; j < Tb; j += 16) out[j] = j;
+                for (int j = hl; j < Tb; j += 16) csr_put(out, j, j, rs, mg.col_capacity);
                 if (hl == 0) { args.row_start[row_id] = (int32_t)rs; args.row_count[row_id] = Tb; }
                 continue;
             }
@@ -1070,8 +1070,8 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
                 while (v) { const int b = __ffs(v) - 1; v &= v - 1; hstage[p++] = 32 * (4 * hl + q) + b; }
             }
             __syncwarp(hmask);
-            for (int p2 = hl; p2 < nk; p2 += 16) out[p2] = hstage[p2];
-            for (int j = sf + hl; j < Tb; j += 16) out[nk + (j - sf)] = j;
+            for (int p2 = hl; p2 < nk; p2 += 16) csr_put(out, p2, hstage[p2], rs, mg.col_capacity);
+            for (int j = sf + hl; j < Tb; j += 16) csr_put(out, nk + (j - sf), j, rs, mg.col_capacity);
             if (hl == 0) { args.row_start[row_id] = (int32_t)rs; args.row_count[row_id] = nk + (Tb - sf); }
             __syncwarp(hmask);
         }

@@ -15,6 +15,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librf2.so")
+CHECKED_LIB_PATH = os.path.join(_HERE, "librf2_checked.so")     # built with RF2_CHECKED=1
 
 RF2_OK = 0
 RF2_ERR_INVALID_ARGUMENT = 1
@@ -22,6 +23,7 @@ RF2_ERR_UNSUPPORTED = 2
 RF2_ERR_INSUFFICIENT_WORKSPACE = 3
 RF2_ERR_CUDA = 4
 RF2_ERR_TIMEOUT = 5
+RF2_ERR_RANGE = 6
 
 # Every entry point declared in include/rf2.h.
 EXPORTED = (
@@ -64,31 +66,46 @@ def lib():
     """Load librf2.so (raises if it has not been built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"CUDA library not built: {LIB_PATH} (run image_dits_b200.build.build())")
-        L = ctypes.CDLL(LIB_PATH)
-        vp, i32, f64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
-        G = ctypes.POINTER(Geometry)
-        L.rf2_status_string.argtypes = [i32]
-        L.rf2_status_string.restype = ctypes.c_char_p
-        L.rf2_query.argtypes = [G, f64, ctypes.POINTER(Sizes)]
-        L.rf2_permutation_index.argtypes = [G, vp]
-        L.rf2_permute.argtypes = [G, vp, vp, vp]
-        L.rf2_unpermute.argtypes = [G, vp, vp, vp]
-        L.rf2_predict_mask.argtypes = [G, vp, vp, f64, vp, vp, vp, vp, sz, vp]
-        L.rf2_predict_mask_static.argtypes = [G, vp, vp, f64, vp, vp, vp, vp]
-        L.rf2_permute_qk_pool.argtypes = [G, vp, vp, vp, vp, vp, sz, vp]
-        L.rf2_predict_mask_pooled.argtypes = [G, f64, vp, vp, vp, vp, sz, vp]
-        L.rf2_predict_mask_cdf.argtypes = [G, vp, vp, f64, vp, vp, vp, vp, sz, vp]
-        L.rf2_predict_mask_cdf_pooled.argtypes = [G, f64, vp, vp, vp, vp, sz, vp]
-        L.rf2_block_sparse_attn.argtypes = [G, vp, vp, vp, vp, vp, vp, vp, vp, vp]
-        L.rf2_device_status.argtypes = [vp]
-        L.rf2_selftest_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.POINTER(ctypes.c_int32), vp]
-        for name in EXPORTED:
-            if name != "rf2_status_string":
-                getattr(L, name).restype = i32
-        _lib = L
+        _lib = load(LIB_PATH)
     return _lib
+
+
+def use_library(path: str):
+    """Route every call of this module through the library at `path` (for
+    example CHECKED_LIB_PATH); returns the one it replaces (None if none was
+    loaded yet)."""
+    global _lib
+    old = _lib
+    _lib = load(path)
+    return old
+
+
+def load(path: str):
+    """Load a build of the library and declare its entry points."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} (run image_dits_b200.build.build())")
+    L = ctypes.CDLL(path)
+    vp, i32, f64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
+    G = ctypes.POINTER(Geometry)
+    L.rf2_status_string.argtypes = [i32]
+    L.rf2_status_string.restype = ctypes.c_char_p
+    L.rf2_query.argtypes = [G, f64, ctypes.POINTER(Sizes)]
+    L.rf2_permutation_index.argtypes = [G, vp]
+    L.rf2_permute.argtypes = [G, vp, vp, vp]
+    L.rf2_unpermute.argtypes = [G, vp, vp, vp]
+    L.rf2_predict_mask.argtypes = [G, vp, vp, f64, vp, vp, vp, vp, sz, vp]
+    L.rf2_predict_mask_static.argtypes = [G, vp, vp, f64, vp, vp, vp, vp]
+    L.rf2_permute_qk_pool.argtypes = [G, vp, vp, vp, vp, vp, sz, vp]
+    L.rf2_predict_mask_pooled.argtypes = [G, f64, vp, vp, vp, vp, sz, vp]
+    L.rf2_predict_mask_cdf.argtypes = [G, vp, vp, f64, vp, vp, vp, vp, sz, vp]
+    L.rf2_predict_mask_cdf_pooled.argtypes = [G, f64, vp, vp, vp, vp, sz, vp]
+    L.rf2_block_sparse_attn.argtypes = [G, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.rf2_device_status.argtypes = [vp]
+    L.rf2_selftest_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.POINTER(ctypes.c_int32), vp]
+    for name in EXPORTED:
+        if name != "rf2_status_string":
+            getattr(L, name).restype = i32
+    return L
 
 
 def status_string(status: int) -> str:

@@ -49,7 +49,9 @@ typedef enum {
     RF2_ERR_UNSUPPORTED = 2,          /* head_dim not 64/128, block not 64, too many blocks */
     RF2_ERR_INSUFFICIENT_WORKSPACE = 3,
     RF2_ERR_CUDA = 4,                 /* a CUDA runtime call or launch failed */
-    RF2_ERR_TIMEOUT = 5               /* a kernel's bounded wait ran out (device status) */
+    RF2_ERR_TIMEOUT = 5,              /* a kernel's bounded wait ran out (device status) */
+    RF2_ERR_RANGE = 6                 /* librf2_checked.so only: an index out of range was
+                                         skipped (device status) */
 } rf2_status;
 
 /* Problem geometry.  The window (win_t, win_h, win_w) is the 3D (video) or 2D
@@ -221,8 +223,18 @@ int rf2_block_sparse_attn(const rf2_geometry* geom, const void* qp_bf16, const v
                           const int32_t* col_idx, void* op_bf16, float* lse, void* stream);
 
 /* Synchronizes `stream`, then returns and clears the device status word of
- * the calling thread's current device: RF2_OK, or RF2_ERR_TIMEOUT if a
- * kernel's bounded wait ran out since the last call. */
+ * the calling thread's current device: RF2_OK, RF2_ERR_TIMEOUT if a kernel's
+ * bounded wait ran out since the last call, or (checked library only, ahead
+ * of a timeout) RF2_ERR_RANGE if a range check failed.
+ *
+ * The checked library, librf2_checked.so, is this library compiled with
+ * RF2_CHECKED=1: the same entry points and results, plus range checks in the
+ * kernels, each of which, when it fails, records RF2_ERR_RANGE here and skips
+ * the access: the CSR rows the attention reads (row_count in [0, T_b],
+ * row_start >= 0 and row_start + row_count within B*H*T_b^2, the largest
+ * layout the library writes; col_idx values in [0, T_b)), every col_idx
+ * store of the mask kernels against the mask's col_idx_capacity, and every
+ * computed permutation source row against [0, N). */
 int rf2_device_status(void* stream);
 
 /* Self-test of failure detection (tests only).  Launches, on `stream`, one
