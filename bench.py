@@ -526,7 +526,8 @@ def main():
         line["e2e"] = {"value": flops_all / (e2e_ms_all * 1e-3) / 1e12, "unit": "TFLOP/s",
                        "ms_per_step": e2e_ms_all, "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                        "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
-                       "api": f"rf2.HostPipeline, {e2e['chunks']} head chunks, copies overlapped with compute"}
+                       "api": f"rf2_attention_host (C ABI, through rf2.HostPipeline), {e2e['chunks']} head chunks, "
+                              "copies overlapped with compute"}
 
     # mask prediction as one call on the permuted Q/K (Q and K read again), for its HBM roofline
     predict = ((lambda: rf2.predict_mask_cdf(g, qp, kp, args.tau, mask, ws)) if args.tau is not None

@@ -856,6 +856,215 @@ int rf2_selftest_wait_timeout(uint32_t limit_us, int32_t* waits_given_up, void* 
     return cudaStreamSynchronize(s) == cudaSuccess ? RF2_OK : RF2_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- host-memory call
+// Heads per chunk: `chunks` near-equal chunks (cuts at round-half-even of
+// c * heads / chunks), the last split into halves (rounded up) down to one head.
+static int host_chunk_sizes(int32_t heads, int32_t chunks, int32_t* sizes, int cap)
+{
+    const int n = (int)(chunks < 1 ? 1 : (chunks > heads ? heads : chunks));
+    int m = 0;
+    int prev = 0;
+    for (int c = 1; c <= n; ++c) {
+        const int cut = (int)nearbyint((double)c * heads / n);
+        if (m >= cap) return -1;
+        sizes[m++] = cut - prev;
+        prev = cut;
+    }
+    int r = sizes[--m];
+    while (r > 1) {
+        const int h = (r + 1) / 2;
+        if (m >= cap) return -1;
+        sizes[m++] = h;
+        r -= h;
+    }
+    if (r) {
+        if (m >= cap) return -1;
+        sizes[m++] = r;
+    }
+    return m;
+}
+
+struct HostPlan {
+    Checked c;
+    int32_t sizes[256];
+    int n;
+    int32_t hmax;
+    rf2_geometry gmax;       // geometry of the largest chunk
+    rf2_sizes sz;            // its mask sizes
+    size_t tensor_bytes, chunk_bytes, work_bytes;
+    size_t off_q, off_k, off_v, off_o, off_qp, off_kp, off_vp, off_op, off_rs, off_rc, off_ci, off_ws;
+};
+
+static rf2_geometry chunk_geometry(const rf2_geometry* g, int32_t heads)
+{
+    rf2_geometry h = *g;
+    h.batch = 1;
+    h.heads = heads;
+    return h;
+}
+
+static int host_plan(const rf2_geometry* geom, double keep, double tau, int32_t chunks, HostPlan& p)
+{
+    p.c = check_geometry(geom);
+    if (p.c.status != RF2_OK) return p.c.status;
+    if ((keep > 0.0) == (tau > 0.0)) return RF2_ERR_INVALID_ARGUMENT;          // exactly one selection
+    if (tau > 0.0 && !(tau <= 1.0)) return RF2_ERR_INVALID_ARGUMENT;
+    if (p.c.BH > INT32_MAX) return RF2_ERR_UNSUPPORTED;
+    p.n = host_chunk_sizes((int32_t)p.c.BH, chunks, p.sizes, 256);
+    if (p.n <= 0) return RF2_ERR_INVALID_ARGUMENT;
+    p.hmax = 0;
+    for (int i = 0; i < p.n; ++i) p.hmax = p.sizes[i] > p.hmax ? p.sizes[i] : p.hmax;
+    p.gmax = chunk_geometry(geom, p.hmax);
+    Checked cm;
+    MaskGeo mg;
+    const int st = sizes_for(&p.gmax, tau > 0.0 ? 1.0 : keep, cm, mg, &p.sz);
+    if (st != RF2_OK) return st;
+    const size_t row_bytes = (size_t)p.c.N * p.c.D * 2;
+    p.tensor_bytes = (size_t)p.c.BH * row_bytes;
+    p.chunk_bytes = (size_t)p.hmax * row_bytes;
+    size_t at = 0;
+    auto take = [&](size_t bytes) { const size_t o = at; at += round256(bytes); return o; };
+    p.off_q = take(p.tensor_bytes);
+    p.off_k = take(p.tensor_bytes);
+    p.off_v = take(p.tensor_bytes);
+    p.off_o = take(p.tensor_bytes);
+    p.off_qp = take(p.chunk_bytes);
+    p.off_kp = take(p.chunk_bytes);
+    p.off_vp = take(p.chunk_bytes);
+    p.off_op = take(p.chunk_bytes);
+    p.off_rs = take((size_t)p.sz.num_rows * 4);
+    p.off_rc = take((size_t)p.sz.num_rows * 4);
+    p.off_ci = take((size_t)p.sz.col_idx_capacity * 4);
+    p.off_ws = take(p.sz.mask_workspace_bytes);
+    p.work_bytes = at;
+    return RF2_OK;
+}
+
+int rf2_attention_host_query(const rf2_geometry* geom, double keep_ratio, double tau, int32_t chunks,
+                             rf2_host_sizes* out)
+{
+    if (!out) return RF2_ERR_INVALID_ARGUMENT;
+    HostPlan p;
+    const int st = host_plan(geom, keep_ratio, tau, chunks, p);
+    if (st != RF2_OK) return st;
+    out->num_chunks = p.n;
+    out->max_chunk_heads = p.hmax;
+    out->work_bytes = p.work_bytes;
+    return RF2_OK;
+}
+
+int rf2_attention_host(const rf2_geometry* geom, double keep_ratio, double tau, int32_t chunks,
+                       const void* q_host, const void* k_host, const void* v_host, void* o_host, void* work,
+                       size_t work_bytes, void* stream_h2d, void* stream_compute, void* stream_d2h,
+                       void** events, int32_t num_events)
+{
+    HostPlan p;
+    int st = host_plan(geom, keep_ratio, tau, chunks, p);
+    if (st != RF2_OK) return st;
+    if (!q_host || !k_host || !v_host || !o_host || !work) return RF2_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q_host) || !aligned16(k_host) || !aligned16(v_host) || !aligned16(o_host) ||
+        (reinterpret_cast<uintptr_t>(work) & 255u))
+        return RF2_ERR_INVALID_ARGUMENT;
+    if (work_bytes < p.work_bytes) return RF2_ERR_INSUFFICIENT_WORKSPACE;
+    cudaStream_t sh = reinterpret_cast<cudaStream_t>(stream_h2d);
+    cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream_compute);
+    cudaStream_t sd = reinterpret_cast<cudaStream_t>(stream_d2h);
+    if (sh == sc || sh == sd || sc == sd) return RF2_ERR_INVALID_ARGUMENT;
+    const bool per_chunk = events != nullptr && num_events > 0;
+    if (per_chunk && num_events < 2 * p.n) return RF2_ERR_INVALID_ARGUMENT;
+    cudaEvent_t* chunk_ev = reinterpret_cast<cudaEvent_t*>(events);   // [2c]: computed, [2c+1]: copied back
+    uint8_t* w = reinterpret_cast<uint8_t*>(work);
+    const size_t row_bytes = (size_t)p.c.N * p.c.D * 2;
+    // events: 0 compute idle, 1 copy-back idle, then per chunk: inputs in, chunk computed
+    const int nev = 2 + 2 * p.n;
+    cudaEvent_t ev[2 + 2 * 256];
+    int made = 0;
+    auto cleanup = [&](int r) {
+        for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+        return r;
+    };
+    clear_pending_error();
+    for (; made < nev; ++made)
+        if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) return cleanup(RF2_ERR_CUDA);
+    // the previous calls on these streams: computation done before `work` is overwritten by
+    // copies, copy-back done before it is overwritten by computation (whole calls, or chunk
+    // by chunk through the caller's events; an event never recorded is no wait)
+    if (!per_chunk &&
+        (cudaEventRecord(ev[0], sc) != cudaSuccess || cudaStreamWaitEvent(sh, ev[0], 0) != cudaSuccess ||
+         cudaEventRecord(ev[1], sd) != cudaSuccess || cudaStreamWaitEvent(sc, ev[1], 0) != cudaSuccess))
+        return cleanup(RF2_ERR_CUDA);
+    // inputs, chunk by chunk
+    int64_t h0 = 0;
+    for (int c = 0; c < p.n; ++c) {
+        const size_t off = (size_t)h0 * row_bytes, bytes = (size_t)p.sizes[c] * row_bytes;
+        if (per_chunk && cudaStreamWaitEvent(sh, chunk_ev[2 * c], 0) != cudaSuccess) return cleanup(RF2_ERR_CUDA);
+        if (cudaMemcpyAsync(w + p.off_q + off, static_cast<const uint8_t*>(q_host) + off, bytes,
+                            cudaMemcpyHostToDevice, sh) != cudaSuccess ||
+            cudaMemcpyAsync(w + p.off_k + off, static_cast<const uint8_t*>(k_host) + off, bytes,
+                            cudaMemcpyHostToDevice, sh) != cudaSuccess ||
+            cudaMemcpyAsync(w + p.off_v + off, static_cast<const uint8_t*>(v_host) + off, bytes,
+                            cudaMemcpyHostToDevice, sh) != cudaSuccess ||
+            cudaEventRecord(ev[2 + 2 * c], sh) != cudaSuccess)
+            return cleanup(RF2_ERR_CUDA);
+        h0 += p.sizes[c];
+    }
+    // computation on one stream (the chunk buffers are reused), each chunk's copy-back after it
+    int32_t* rs = reinterpret_cast<int32_t*>(w + p.off_rs);
+    int32_t* rc = reinterpret_cast<int32_t*>(w + p.off_rc);
+    int32_t* ci = reinterpret_cast<int32_t*>(w + p.off_ci);
+    void* ws = w + p.off_ws;
+    h0 = 0;
+    for (int c = 0; c < p.n; ++c) {
+        const rf2_geometry g = chunk_geometry(geom, p.sizes[c]);
+        const size_t off = (size_t)h0 * row_bytes, bytes = (size_t)p.sizes[c] * row_bytes;
+        if (cudaStreamWaitEvent(sc, ev[2 + 2 * c], 0) != cudaSuccess ||
+            (per_chunk && cudaStreamWaitEvent(sc, chunk_ev[2 * c + 1], 0) != cudaSuccess))
+            return cleanup(RF2_ERR_CUDA);
+        st = rf2_permute_qk_pool(&g, w + p.off_q + off, w + p.off_k + off, w + p.off_qp, w + p.off_kp, ws,
+                                 p.sz.mask_workspace_bytes, sc);
+        if (st == RF2_OK) st = rf2_permute(&g, w + p.off_v + off, w + p.off_vp, sc);
+        if (st == RF2_OK)
+            st = (tau > 0.0) ? rf2_predict_mask_cdf_pooled(&g, tau, rs, rc, ci, ws, p.sz.mask_workspace_bytes, sc)
+                             : rf2_predict_mask_pooled(&g, keep_ratio, rs, rc, ci, ws, p.sz.mask_workspace_bytes, sc);
+        if (st == RF2_OK)
+            st = rf2_block_sparse_attn(&g, w + p.off_qp, w + p.off_kp, w + p.off_vp, rs, rc, ci, w + p.off_op,
+                                       nullptr, sc);
+        if (st == RF2_OK) st = rf2_unpermute(&g, w + p.off_op, w + p.off_o + off, sc);
+        if (st != RF2_OK) return cleanup(st);
+        if (cudaEventRecord(ev[3 + 2 * c], sc) != cudaSuccess || cudaStreamWaitEvent(sd, ev[3 + 2 * c], 0) != cudaSuccess ||
+            (per_chunk && cudaEventRecord(chunk_ev[2 * c], sc) != cudaSuccess) ||
+            cudaMemcpyAsync(static_cast<uint8_t*>(o_host) + off, w + p.off_o + off, bytes, cudaMemcpyDeviceToHost,
+                            sd) != cudaSuccess ||
+            (per_chunk && cudaEventRecord(chunk_ev[2 * c + 1], sd) != cudaSuccess))
+            return cleanup(RF2_ERR_CUDA);
+        h0 += p.sizes[c];
+    }
+    return cleanup(RF2_OK);
+}
+
+int rf2_host_events_create(int32_t count, void** events)
+{
+    if (count < 0 || (count > 0 && !events)) return RF2_ERR_INVALID_ARGUMENT;
+    for (int32_t i = 0; i < count; ++i) {
+        cudaEvent_t e;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+            for (int32_t k = 0; k < i; ++k) cudaEventDestroy(reinterpret_cast<cudaEvent_t>(events[k]));
+            return RF2_ERR_CUDA;
+        }
+        events[i] = e;
+    }
+    return RF2_OK;
+}
+
+int rf2_host_events_destroy(int32_t count, void** events)
+{
+    if (count < 0 || (count > 0 && !events)) return RF2_ERR_INVALID_ARGUMENT;
+    int st = RF2_OK;
+    for (int32_t i = 0; i < count; ++i)
+        if (events[i] && cudaEventDestroy(reinterpret_cast<cudaEvent_t>(events[i])) != cudaSuccess) st = RF2_ERR_CUDA;
+    return st;
+}
+
 int rf2_device_status(void* stream)
 {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -31,6 +31,7 @@ EXPORTED = (
     "rf2_predict_mask", "rf2_predict_mask_static", "rf2_permute_qk_pool", "rf2_predict_mask_pooled",
     "rf2_predict_mask_cdf", "rf2_predict_mask_cdf_pooled",
     "rf2_block_sparse_attn", "rf2_device_status", "rf2_selftest_wait_timeout",
+    "rf2_attention_host_query", "rf2_attention_host", "rf2_host_events_create", "rf2_host_events_destroy",
 )
 
 
@@ -102,6 +103,11 @@ def load(path: str):
     L.rf2_block_sparse_attn.argtypes = [G, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.rf2_device_status.argtypes = [vp]
     L.rf2_selftest_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.POINTER(ctypes.c_int32), vp]
+    L.rf2_attention_host_query.argtypes = [G, f64, f64, i32, ctypes.POINTER(HostSizes)]
+    L.rf2_attention_host.argtypes = [G, f64, f64, i32, vp, vp, vp, vp, vp, sz, vp, vp, vp,
+                                     ctypes.POINTER(vp), i32]
+    L.rf2_host_events_create.argtypes = [i32, ctypes.POINTER(vp)]
+    L.rf2_host_events_destroy.argtypes = [i32, ctypes.POINTER(vp)]
     for name in EXPORTED:
         if name != "rf2_status_string":
             getattr(L, name).restype = i32
@@ -335,112 +341,74 @@ def chunk_sizes(heads: int, chunks: int, tail_split: bool = True) -> list:
     return sizes
 
 
+class HostSizes(ctypes.Structure):
+    _fields_ = [("num_chunks", ctypes.c_int32), ("max_chunk_heads", ctypes.c_int32), ("work_bytes", ctypes.c_size_t)]
+
+
+def host_query(geom: Geometry, keep: float | None = None, tau: float | None = None, chunks: int = 8) -> HostSizes:
+    """rf2_attention_host_query: chunk count and device scratch of rf2_attention_host."""
+    out = HostSizes()
+    _check(lib().rf2_attention_host_query(ctypes.byref(geom), float(keep or 0.0), float(tau or 0.0), int(chunks),
+                                          ctypes.byref(out)), "rf2_attention_host_query")
+    return out
+
+
 class HostPipeline:
-    """One attention call on host (pinned) tensors, copies overlapped with compute.
+    """One attention call on host (pinned) tensors, copies overlapped with
+    compute: a thin wrapper over the C call rf2_attention_host, which copies
+    head chunks in on one stream, computes them on a second and copies them
+    back on a third (see include/rf2.h).  Output bits equal those of the calls
+    on the whole device tensors.
 
-    The (batch, head) problems of the path are independent (permutation, mask
-    and attention are per head), so the heads are processed in chunks: the
-    host-to-device copy of chunk c + 1 and the device-to-host copy of chunk
-    c - 1 run on their own streams while chunk c is computed.  Every chunk is
-    computed by the same library calls as `rainfusion_attention` on a
-    heads-slice geometry, so the output is bit-identical to the unchunked call.
-
-    Build once (device buffers, streams and masks are allocated here), then
-    call `run(q, k, v, o)` with pinned host bf16 tensors [B, H, N, d].
-    Selection: top-n with `keep`, or the CDF threshold with `tau`.  The heads
-    are split into `chunks` equal chunks, the last of them (with `tail_split`)
-    further into shrinking parts down to one head.
+    Build once (the device scratch and the three streams are allocated here),
+    then call `run(q, k, v, o)` with pinned host bf16 tensors [B, H, N, d].
+    Selection: top-n with `keep`, or the CDF threshold with `tau`.  The B*H
+    heads go in `chunks` near-equal chunks, the last of them further split in
+    shrinking parts down to one head (`chunk_sizes`).
     """
 
     def __init__(self, geom: Geometry, keep: float | None = None, tau: float | None = None, chunks: int = 8,
-                 device=None, tail_split: bool = True):
+                 device=None, chunk_events: bool = True):
         if (keep is None) == (tau is None):
             raise ValueError("give exactly one of keep and tau")
-        self.geom, self.keep, self.tau = geom, keep, tau
+        self.geom, self.keep, self.tau, self.chunks = geom, keep, tau, int(chunks)
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         self.device = dev
-        BH = geom.batch * geom.heads
-        sizes = chunk_sizes(BH, chunks, tail_split)
-        cuts = [0]
-        for sz in sizes:
-            cuts.append(cuts[-1] + sz)
-        self.parts = []
-        for c in range(len(sizes)):
-            h0, h1 = cuts[c], cuts[c + 1]
-            g = make_geometry(1, h1 - h0, geom.head_dim, geom.frames, geom.height, geom.width, geom.win_t,
-                              geom.win_h, geom.win_w, geom.first_frame_sink, geom.block, geom.text_tokens)
-            self.parts.append((h0, h1, g))
-        N, d = num_tokens(geom), geom.head_dim
-        self.shape = (geom.batch, geom.heads, N, d)
-        hmax = max(h1 - h0 for h0, h1, _ in self.parts)
-        mk = lambda rows: torch.empty((rows, N, d), dtype=torch.bfloat16, device=dev)
-        self.q, self.k, self.v, self.o = mk(BH), mk(BH), mk(BH), mk(BH)
-        self.qp, self.kp, self.vp, self.op = mk(hmax), mk(hmax), mk(hmax), mk(hmax)
-        self.masks = {}
-        for _, _, g in self.parts:
-            if g.heads not in self.masks:
-                self.masks[g.heads] = alloc_mask(g, keep if tau is None else 1.0, dev)
+        sz = host_query(geom, keep, tau, self.chunks)
+        self.parts = chunk_sizes(geom.batch * geom.heads, self.chunks)
+        assert len(self.parts) == sz.num_chunks and max(self.parts) == sz.max_chunk_heads
+        self.work = torch.empty(max(256, sz.work_bytes), dtype=torch.uint8, device=dev)
+        self.shape = (geom.batch, geom.heads, num_tokens(geom), geom.head_dim)
         self.h2d, self.comp, self.d2h = (torch.cuda.Stream(device=dev) for _ in range(3))
-        self.in_ready = [torch.cuda.Event() for _ in self.parts]
-        self.done = [torch.cuda.Event() for _ in self.parts]
-        self.out_read = [torch.cuda.Event() for _ in self.parts]
-        self.runs = 0
+        # chunk-by-chunk ordering of consecutive runs (chunk c waits only for chunk c of the
+        # last run); without, each run waits for the whole previous one
+        self.num_events = 2 * sz.num_chunks if chunk_events else 0
+        self.events = (ctypes.c_void_p * self.num_events)() if chunk_events else None
+        if chunk_events:
+            with torch.cuda.device(dev):
+                _check(lib().rf2_host_events_create(self.num_events, self.events), "rf2_host_events_create")
+        self._lib = lib()
+
+    def __del__(self):
+        events = getattr(self, "events", None)
+        if events is not None:
+            try:
+                self.d2h.synchronize()
+                self._lib.rf2_host_events_destroy(self.num_events, events)
+            except Exception:
+                pass
 
     def run(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor, o_host: torch.Tensor):
         for t in (q_host, k_host, v_host, o_host):
             if not (t.device.type == "cpu" and t.is_pinned() and t.dtype == torch.bfloat16 and t.is_contiguous()
                     and tuple(t.shape) == self.shape):
                 raise ValueError(f"expected pinned contiguous host bf16 tensors of shape {self.shape}")
-        N, d = self.shape[2], self.shape[3]
-        hq, hk, hv, ho = (t.view(-1, N, d) for t in (q_host, k_host, v_host, o_host))
-        first = self.runs == 0
-        # inputs: the previous run's computation of a chunk must be done with its device copies
-        with torch.cuda.stream(self.h2d):
-            for c, (h0, h1, _) in enumerate(self.parts):
-                if not first:
-                    self.h2d.wait_event(self.done[c])
-                self.q[h0:h1].copy_(hq[h0:h1], non_blocking=True)
-                self.k[h0:h1].copy_(hk[h0:h1], non_blocking=True)
-                self.v[h0:h1].copy_(hv[h0:h1], non_blocking=True)
-                self.in_ready[c].record(self.h2d)
-        # compute, chunk by chunk, on one stream (the work buffers are reused)
-        for c, (h0, h1, g) in enumerate(self.parts):
-            self.comp.wait_event(self.in_ready[c])
-            if not first:
-                self.comp.wait_event(self.out_read[c])       # the previous run's read of this chunk of o
-            m = h1 - h0
-            mask, ws = self.masks[m]
-            qp, kp, vp, op = self.qp[:m], self.kp[:m], self.vp[:m], self.op[:m]
-            s = self.comp
-            _check(lib().rf2_permute_qk_pool(ctypes.byref(g), self.q[h0:h1].data_ptr(), self.k[h0:h1].data_ptr(),
-                                             qp.data_ptr(), kp.data_ptr(), ws.data_ptr(), ws.numel(),
-                                             s.cuda_stream), "rf2_permute_qk_pool")
-            _check(lib().rf2_permute(ctypes.byref(g), self.v[h0:h1].data_ptr(), vp.data_ptr(), s.cuda_stream),
-                   "rf2_permute")
-            if self.tau is None:
-                _check(lib().rf2_predict_mask_pooled(ctypes.byref(g), float(self.keep), mask.row_start.data_ptr(),
-                                                     mask.row_count.data_ptr(), mask.col_idx.data_ptr(),
-                                                     ws.data_ptr(), ws.numel(), s.cuda_stream),
-                       "rf2_predict_mask_pooled")
-            else:
-                _check(lib().rf2_predict_mask_cdf_pooled(ctypes.byref(g), float(self.tau),
-                                                         mask.row_start.data_ptr(), mask.row_count.data_ptr(),
-                                                         mask.col_idx.data_ptr(), ws.data_ptr(), ws.numel(),
-                                                         s.cuda_stream), "rf2_predict_mask_cdf_pooled")
-            _check(lib().rf2_block_sparse_attn(ctypes.byref(g), qp.data_ptr(), kp.data_ptr(), vp.data_ptr(),
-                                               mask.row_start.data_ptr(), mask.row_count.data_ptr(),
-                                               mask.col_idx.data_ptr(), op.data_ptr(), None, s.cuda_stream),
-                   "rf2_block_sparse_attn")
-            _check(lib().rf2_unpermute(ctypes.byref(g), op.data_ptr(), self.o[h0:h1].data_ptr(), s.cuda_stream),
-                   "rf2_unpermute")
-            self.done[c].record(self.comp)
-        # outputs
-        with torch.cuda.stream(self.d2h):
-            for c, (h0, h1, _) in enumerate(self.parts):
-                self.d2h.wait_event(self.done[c])
-                ho[h0:h1].copy_(self.o[h0:h1], non_blocking=True)
-                self.out_read[c].record(self.d2h)
-        self.runs += 1
+        _check(lib().rf2_attention_host(ctypes.byref(self.geom), float(self.keep or 0.0), float(self.tau or 0.0),
+                                        self.chunks, q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
+                                        o_host.data_ptr(), self.work.data_ptr(), self.work.numel(),
+                                        self.h2d.cuda_stream, self.comp.cuda_stream, self.d2h.cuda_stream,
+                                        self.events, self.num_events),
+               "rf2_attention_host")
         return o_host
 
     def synchronize(self):

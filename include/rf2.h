@@ -222,6 +222,58 @@ int rf2_block_sparse_attn(const rf2_geometry* geom, const void* qp_bf16, const v
                           const void* vp_bf16, const int32_t* row_start, const int32_t* row_count,
                           const int32_t* col_idx, void* op_bf16, float* lse, void* stream);
 
+/* One attention call on HOST memory, end to end: the host-to-device copy of
+ * Q, K, V, the whole path (rf2_permute_qk_pool, rf2_permute of V,
+ * rf2_predict_mask_pooled or rf2_predict_mask_cdf_pooled, rf2_block_sparse_attn,
+ * rf2_unpermute) and the device-to-host copy of O.  The (batch, head) problems
+ * are independent (sections 3.1-3.4 are all per head), so the B*H heads go in
+ * chunks: `chunks` near-equal ones, the last split further into shrinking
+ * parts down to one head (what follows the last input copy is then small).
+ * Chunk c's input copies run on stream_h2d, its computation on
+ * stream_compute, its output copy on stream_d2h; the copies of one chunk
+ * overlap the computation of another.  Each chunk is computed by the same
+ * calls on a geometry of its heads, so O is bit-identical to the calls on the
+ * whole tensors.
+ *   keep_ratio, tau   exactly one > 0: top-n selection with keep_ratio, or
+ *                     the CDF threshold with tau (both in (0, 1])
+ *   q/k/v/o_host      bf16 [B, H, N, d] in page-locked host memory (16-byte
+ *                     aligned); o_host is written
+ *   work              device scratch of at least rf2_attention_host_query's
+ *                     work_bytes (256-byte aligned); the library allocates
+ *                     no memory (it creates and destroys a few CUDA events)
+ *   stream_*          three streams (may not be the same stream twice)
+ *   events, num_events  NULL / 0, or 2 * num_chunks events from
+ *                     rf2_host_events_create, the same array on every call
+ *                     with this `work` (see below)
+ * Returns after enqueueing: the host buffers and `work` must stay untouched
+ * until stream_d2h has completed.  Calls one after another on the same
+ * `work` are ordered: without events, a call's copies wait for everything
+ * already on stream_compute and its computation for everything already on
+ * stream_d2h; with events, chunk c of a call waits only for chunk c of the
+ * previous call (its computation before the copy into the chunk's inputs,
+ * its copy-back before the computation into the chunk's output), so the
+ * input copies of the next call start while the previous one computes.
+ * Errors as the calls it makes; after an error part of the work may be
+ * enqueued. */
+typedef struct {
+    int32_t num_chunks;      /* chunks after the tail split */
+    int32_t max_chunk_heads; /* heads of the largest chunk */
+    size_t  work_bytes;      /* device scratch rf2_attention_host needs */
+} rf2_host_sizes;
+
+int rf2_attention_host_query(const rf2_geometry* geom, double keep_ratio, double tau, int32_t chunks,
+                             rf2_host_sizes* out);
+int rf2_attention_host(const rf2_geometry* geom, double keep_ratio, double tau, int32_t chunks,
+                       const void* q_host, const void* k_host, const void* v_host, void* o_host, void* work,
+                       size_t work_bytes, void* stream_h2d, void* stream_compute, void* stream_d2h,
+                       void** events, int32_t num_events);
+
+/* `count` CUDA events (timing disabled) for rf2_attention_host, created on
+ * the current device into events[0 .. count); destroy them with
+ * rf2_host_events_destroy once no enqueued call uses them. */
+int rf2_host_events_create(int32_t count, void** events);
+int rf2_host_events_destroy(int32_t count, void** events);
+
 /* Synchronizes `stream`, then returns and clears the device status word of
  * the calling thread's current device: RF2_OK, RF2_ERR_TIMEOUT if a kernel's
  * bounded wait ran out since the last call, or (checked library only, ahead

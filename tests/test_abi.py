@@ -220,6 +220,35 @@ def test_host_pipeline_chunk_sizes():
     assert rf2.chunk_sizes(40, 8) == [5, 5, 5, 5, 5, 5, 5, 3, 1, 1]
 
 
+def test_host_call_plan(L):
+    """rf2_attention_host_query (host only): the C chunking equals
+    rf2.chunk_sizes (cuts at round-half-even of c*heads/chunks, the last chunk
+    halved down to one head), and the device scratch is the four whole
+    tensors, four chunk tensors of the largest chunk and its mask and mask
+    workspace, each rounded up to 256 bytes; bad selections are refused."""
+    import dataclasses
+    r256 = lambda b: (b + 255) // 256 * 256
+    for name, heads, chunks, keep, tau in [("video720p", 40, 8, 0.2, None), ("image", 24, 5, 0.5, None),
+                                          ("video480p", 12, 3, None, 0.2), ("tiny", 2, 7, 0.5, None),
+                                          ("video480p", 5, 2, 0.2, None)]:
+        wl = dataclasses.replace(WORKLOADS[name], heads=heads)
+        g = rf2.geometry_of(wl)
+        hs = rf2.host_query(g, keep, tau, chunks)
+        parts = rf2.chunk_sizes(heads, chunks)
+        assert hs.num_chunks == len(parts) and hs.max_chunk_heads == max(parts)
+        gm = rf2.geometry_of(dataclasses.replace(wl, heads=max(parts)))
+        sz = rf2.query(gm, 1.0 if tau else keep)
+        row = wl.num_tokens * wl.head_dim * 2
+        want = (4 * r256(heads * row) + 4 * r256(max(parts) * row) + 2 * r256(4 * sz.num_rows)
+                + r256(4 * sz.col_idx_capacity) + r256(sz.mask_workspace_bytes))
+        assert hs.work_bytes == want, (name, hs.work_bytes, want)
+    g = rf2.geometry_of(WORKLOADS["tiny"])
+    out = rf2.HostSizes()
+    for keep, tau in [(0.0, 0.0), (0.5, 0.5), (0.0, 1.5), (-1.0, 0.0)]:
+        assert L.rf2_attention_host_query(ctypes.byref(g), keep, tau, 4, ctypes.byref(out)) == rf2.RF2_ERR_INVALID_ARGUMENT
+    assert L.rf2_attention_host_query(ctypes.byref(g), 0.5, 0.0, 4, None) == rf2.RF2_ERR_INVALID_ARGUMENT
+
+
 def test_static_scratch_size_limit_on_host(L):
     """rf2_predict_mask_static refuses, on the host and before any device call,
     a problem whose block means (hi/lo pair) plus one head's pooled scores

@@ -330,11 +330,36 @@ def test_device_status_clean():
     assert rf2.device_status() == rf2.RF2_OK
 
 
+@pytest.mark.parametrize("chunk_events", [True, False])
+def test_host_call_back_to_back(chunk_events):
+    """rf2_attention_host called twice in a row on different inputs without a
+    synchronization between: the second call's copies wait for the first
+    call's computation (chunk by chunk with the caller's events, else as a
+    whole), so both outputs equal their device-path results."""
+    wl = WORKLOADS["video480p"]
+    g = rf2.geometry_of(wl)
+    refs, hosts = [], []
+    for seed in (8, 9):
+        q, k, v = make_qkv(wl, "cuda", seed=seed)
+        ref, _ = rf2.rainfusion_attention(g, q, k, v, wl.keep)
+        refs.append(ref.cpu())
+        hosts.append(tuple(x.cpu().pin_memory() for x in (q, k, v)) + (torch.empty_like(q, device="cpu").pin_memory(),))
+    torch.cuda.synchronize()
+    pipe = rf2.HostPipeline(g, keep=wl.keep, chunks=4, chunk_events=chunk_events)
+    for hq, hk, hv, ho in hosts:
+        pipe.run(hq, hk, hv, ho)
+    pipe.synchronize()
+    for (hq, hk, hv, ho), ref in zip(hosts, refs):
+        assert torch.equal(ho.view(torch.int16), ref.view(torch.int16))
+    assert rf2.device_status() == rf2.RF2_OK
+
+
 @pytest.mark.parametrize("name,chunks,tau", [("tiny", 2, None), ("image", 5, None), ("video480p_text", 4, None),
                                              ("video480p", 3, 0.2)])
 def test_host_pipeline_matches_device_path(name, chunks, tau):
-    """HostPipeline (head chunks, copies overlapped with compute) gives the same
-    output bits as the single device call, over two back-to-back runs."""
+    """rf2_attention_host through HostPipeline (head chunks, copies overlapped
+    with compute) gives the same output bits as the single device call, over
+    two runs."""
     wl = WORKLOADS[name]
     q, k, v = make_qkv(wl, "cuda", seed=4)
     g = rf2.geometry_of(wl)
