@@ -22,7 +22,8 @@
 // Roles (256 threads, two CTAs per SM):
 //   warps 0-3  softmax + epilogue: thread r owns query row r = TMEM lane r
 //   warp 4     MMA issuer (one thread)
-//   warp 5     TMA: Q once, then K of the even entries (stage 0)
+//   warp 5     TMA: K of the even entries (stage 0); Q is loaded once by
+//              thread 0 as soon as the barriers exist
 //   warp 6     TMA: K of the odd entries (stage 1)
 //   warp 7     TMA: V of every entry (stage e mod 2)
 // (one thread's TMA stream is served serially, so loads are spread over three
@@ -212,6 +213,9 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_init(smem_u32(&ctl->drain), 1);
         ctl->abort = 0;
         fence_mbar_init();
+        // Q first: its load overlaps the set-up below (the Q region is not touched before)
+        mbar_arrive_expect_tx(smem_u32(&ctl->q_full), Cfg::Q_BYTES);
+        tma_load_4d(base_u32 + Cfg::OFF_Q, &tm_q, smem_u32(&ctl->q_full), 0, qb0 * 64, 0, (int)bh);
     }
     if (warp == Cfg::KA_WARP && lane == 0) {
         prefetch_tmap(&tm_q);
@@ -309,10 +313,6 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (lane == 0) {
             fence_proxy_async_smem();   // the K stages held the row bitmaps (generic accesses)
             const int g = (warp == Cfg::KA_WARP) ? 0 : 1;
-            if (g == 0) {
-                mbar_arrive_expect_tx(smem_u32(&ctl->q_full), Cfg::Q_BYTES);
-                tma_load_4d(base_u32 + Cfg::OFF_Q, &tm_q, smem_u32(&ctl->q_full), 0, qb0 * 64, 0, (int)bh);
-            }
             const uint32_t full = smem_u32(&ctl->k_full[g]);
             const uint32_t dst = base_u32 + Cfg::OFF_K + g * Cfg::KV_BLOCK;
             int issued = -1;
