@@ -197,6 +197,37 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     const int qb0 = 2 * pair;
     const bool has_b = (qb0 + 1) < Tb;
+    const int64_t rA = bh * Tb + qb0;
+
+    // The two CSR rows' extents and first entries (up to 2 x 256 per row),
+    // read into registers before the set-up below so that their two dependent
+    // round trips to memory overlap it.  (Checked build: a row outside the CSR
+    // array, or a key block outside 0 .. T_b - 1, is reported and skipped.)
+    auto row_len = [&](int64_t r) -> int {
+        const int32_t cnt = args.row_count[r];
+        const int len = min(max(cnt, 0), Tb);
+        if (RF2_CHECKED && !in_range(cnt >= 0 && cnt <= Tb && args.row_start[r] >= 0 &&
+                                     (int64_t)args.row_start[r] + cnt <= args.col_capacity))
+            return 0;
+        return len;
+    };
+    int lenA = 0, lenB = 0;
+    const int32_t* srcA = args.col_idx;
+    const int32_t* srcB = args.col_idx;
+    int32_t first[4] = {-1, -1, -1, -1};               // entries tid and tid + 256 of rows A and B
+    auto read_rows = [&]() {
+        lenA = row_len(rA);
+        srcA = args.col_idx + args.row_start[rA];
+        if (has_b) {
+            lenB = row_len(rA + 1);
+            srcB = args.col_idx + args.row_start[rA + 1];
+        }
+        first[0] = (tid < lenA) ? srcA[tid] : -1;
+        first[1] = (tid + Cfg::THREADS < lenA) ? srcA[tid + Cfg::THREADS] : -1;
+        first[2] = (tid < lenB) ? srcB[tid] : -1;
+        first[3] = (tid + Cfg::THREADS < lenB) ? srcB[tid + Cfg::THREADS] : -1;
+    };
+    if (warp != 0) read_rows();
 
     // ---- set-up: barriers, TMEM, union of the two CSR rows
     if (tid == 0) {
@@ -225,6 +256,7 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (warp == 0) {
         tmem_alloc(smem_u32(&ctl->tmem_base), Cfg::TM_COLS);
         tmem_relinquish();
+        read_rows();
     }
     // Union of the two CSR rows as bitmaps (one bit per key block and query
     // block), built in the still unused K stage, then compacted in ascending
@@ -238,32 +270,16 @@ block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
-    const int64_t rA = bh * Tb + qb0;
     {
-        // (checked build: a row outside the CSR array, or a key block outside
-        // 0 .. T_b - 1, is reported and skipped)
-        auto row_len = [&](int64_t r) -> int {
-            const int32_t cnt = args.row_count[r];
-            const int len = min(max(cnt, 0), Tb);
-            if (RF2_CHECKED && !in_range(cnt >= 0 && cnt <= Tb && args.row_start[r] >= 0 &&
-                                         (int64_t)args.row_start[r] + cnt <= args.col_capacity))
-                return 0;
-            return len;
+        auto set_bit = [&](uint32_t* bm, int32_t j) {
+            if (in_range(j >= 0 && j < Tb) && j >= 0 && j < Tb) atomicOr(&bm[j >> 5], 1u << (j & 31));
         };
-        const int lenA = row_len(rA);
-        const int32_t* srcA = args.col_idx + args.row_start[rA];
-        for (int e = tid; e < lenA; e += Cfg::THREADS) {
-            const int32_t j = srcA[e];
-            if (in_range(j >= 0 && j < Tb) && j >= 0 && j < Tb) atomicOr(&bmA[j >> 5], 1u << (j & 31));
-        }
-        if (has_b) {
-            const int lenB = row_len(rA + 1);
-            const int32_t* srcB = args.col_idx + args.row_start[rA + 1];
-            for (int e = tid; e < lenB; e += Cfg::THREADS) {
-                const int32_t j = srcB[e];
-                if (in_range(j >= 0 && j < Tb) && j >= 0 && j < Tb) atomicOr(&bmB[j >> 5], 1u << (j & 31));
-            }
-        }
+        if (tid < lenA) set_bit(bmA, first[0]);
+        if (tid + Cfg::THREADS < lenA) set_bit(bmA, first[1]);
+        if (tid < lenB) set_bit(bmB, first[2]);
+        if (tid + Cfg::THREADS < lenB) set_bit(bmB, first[3]);
+        for (int e = tid + 2 * Cfg::THREADS; e < lenA; e += Cfg::THREADS) set_bit(bmA, srcA[e]);
+        for (int e = tid + 2 * Cfg::THREADS; e < lenB; e += Cfg::THREADS) set_bit(bmB, srcB[e]);
     }
     __syncthreads();
     if (warp == 0) {
