@@ -76,13 +76,13 @@ def kept_flops_from_mask(mask, wl) -> float:
 
 # DRAM bytes (read + write) per (token, head) of one block_sparse_attn_kernel<128>
 # launch: dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture on the
-# 720p shape with 8 heads (513.95 MB + 138.25 MB over 75,600 tokens x 8 heads), of
+# 720p shape with 8 heads (514.98 MB + 137.66 MB over 75,600 tokens x 8 heads), of
 # the kernel as built at ATTN_TRAFFIC_BUILD.  The kernel's DRAM traffic is its
 # compulsory Q/K/V reads and O writes (1,024 B per token-head; K/V re-reads hit L2),
 # so it scales with the token-heads of the workload.  Re-measure whenever the
 # kernel changes.
-ATTN_DRAM_BYTES_PER_TOKEN_HEAD = (513.947904e6 + 138.250496e6) / (75600 * 8)
-ATTN_TRAFFIC_BUILD = "8e078e7"
+ATTN_DRAM_BYTES_PER_TOKEN_HEAD = (514.980864e6 + 137.662464e6) / (75600 * 8)
+ATTN_TRAFFIC_BUILD = "02d6d5b"
 
 
 def mask_bytes(wl, mask) -> float:
