@@ -485,11 +485,10 @@ static int launch_topn(const Checked& c, const MaskGeo& mg, const MaskWs& w, int
         return RF2_ERR_CUDA;
     if (ensure_dynamic_smem(reinterpret_cast<const void*>(topn_codes_kernel<D>), Cfg::SMEM) != RF2_OK)
         return RF2_ERR_CUDA;
-    // topn_rows_kernel: bitmaps [32][G | 1], bin-b* keys [64][32] (then two rows of
-    // up to n_keep kept keys), row kinds [32];
+    // topn_rows_kernel: bitmaps [32][G | 1], bin-b* keys [64][32];
     // topn_overflow_kernel: the keys of the threshold code, their scores, radix bins
     const int G = (c.Tb + 31) / 32;
-    const size_t rows_smem = ((size_t)32 * (G | 1) + (64 * 32 > 2 * mg.n_keep ? 64 * 32 : 2 * mg.n_keep) + 32) * 4;
+    const size_t rows_smem = ((size_t)32 * (G | 1) + 64 * 32) * 4;
     const size_t ovf_smem = (size_t)(2 * c.Tb + 256) * 4;
     if (ensure_dynamic_smem(reinterpret_cast<const void*>(topn_rows_kernel<D>), rows_smem) != RF2_OK ||
         ensure_dynamic_smem(reinterpret_cast<const void*>(topn_overflow_kernel<D>), ovf_smem) != RF2_OK)

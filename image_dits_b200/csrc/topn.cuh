@@ -769,11 +769,9 @@ __global__ void __launch_bounds__(256) topn_overflow_kernel(const TopnArgs args)
 //      64 keys in bin b*, more than 16 keys of c* to rank, more than 4 keys
 //      tied in the fine code, or its threshold in a saturated code (0 or 255:
 //      the bracket missed) is listed for topn_overflow_kernel.
-//   4. Each half-warp writes one row at a time: each lane expands the kept bits
-//      of four bitmap words into shared memory at its offset (a scan of the
-//      words' counts over the half-warp), and the row leaves in 64-byte
-//      stores, the sink columns last; sink rows (and keep = 1) keep every
-//      block.
+//   4. Each thread writes its own row: the kept bits of its bitmap in
+//      ascending order, then the sink columns; sink rows (and keep = 1) keep
+//      every block.  The 32 rows go out in parallel.
 template <int D>
 __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
 {
@@ -790,10 +788,7 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
     const int row_end = min(mg.sink_first, Tb);
     const int sf = mg.sink_first;                          // <= Tb
     uint32_t* bm = reinterpret_cast<uint32_t*>(smem_raw);              // [32][BS]
-    const int SH = max(BCAP * 32, 2 * n) / 2;              // staging entries per half-warp (>= n)
     uint32_t* cand = bm + 32 * BS;                                       // [BCAP][32]: code16 << 16 | j
-    int32_t* stage = reinterpret_cast<int32_t*>(cand);                   // then: [2][SH] rows being written
-    int32_t* kind = reinterpret_cast<int32_t*>(cand + 2 * SH);           // [32]: row kind
     const int64_t units = args.BH * mtiles * 4;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
         const int64_t item = u >> 2;
@@ -1019,61 +1014,36 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
                 args.overflow[1 + at] = (int32_t)(bh * Tb + i);
             }
         }
-        kind[lane] = rk;
-        __syncwarp();
-        // 4. the CSR rows of the warp's 32 query blocks, two at a time: half-warp h
-        // writes rows 16 h + r; lane l of it holds bitmap words 4 l .. 4 l + 3
-        const int wl = (sf + 31) >> 5;                     // bitmap words below the sink columns
-        const int hw = lane >> 4, hl = lane & 15;
-        const unsigned hmask = 0xFFFFu << (16 * hw);
-        int32_t* hstage = stage + hw * SH;
-        #pragma unroll 1
-        for (int r0 = 0; r0 < 16; ++r0) {
-            const int rr = 16 * hw + r0;
-            const int k = kind[rr];
-            if (k >= 2) continue;                              // no row, or the overflow kernel writes it
-            const int ir = m0 + (rl - lane) + rr;
-            const int64_t row_id = bh * Tb + ir;
-            const int64_t rs = row_offset(mg, bh, ir);
+        // 4. the CSR rows: thread r writes row r from its own bitmap (rows stride
+        // BS, odd: the lanes' words sit in distinct banks), kept keys below the
+        // sink columns in ascending order, then the sink columns.  The rows are
+        // written in parallel; each lane's stores run through its row in order.
+        if (rk < 2) {
+            const int64_t row_id = bh * Tb + i;
+            const int64_t rs = row_offset(mg, bh, i);
             int32_t* out = args.col_idx + rs;
-            if (k == 1) {
-                for (int j = hl; j < Tb; j += 16) csr_put(out, j, j, rs, mg.col_capacity);
-                if (hl == 0) { args.row_start[row_id] = (int32_t)rs; args.row_count[row_id] = Tb; }
-                continue;
-            }
-            const uint32_t* brow = bm + rr * BS;
-            uint32_t x[4];
-            int c = 0;
-            #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int wi = 4 * hl + q;
-                uint32_t v = 0u;
-                if (wi < wl) {
-                    v = brow[wi];
+            if (rk == 1) {
+                for (int j = 0; j < Tb; ++j) csr_put(out, j, j, rs, mg.col_capacity);
+                args.row_start[row_id] = (int32_t)rs;
+                args.row_count[row_id] = Tb;
+            } else {
+                const uint32_t* brow = bm + lane * BS;
+                const int wl = (sf + 31) >> 5;             // bitmap words below the sink columns
+                int nk = 0;
+                for (int wi = 0; wi < wl; ++wi) {
+                    uint32_t v = brow[wi];
                     const int j0 = 32 * wi;
                     if (j0 + 32 > sf) v &= (1u << (sf - j0)) - 1u;
+                    while (v) {
+                        const int b = __ffs(v) - 1;
+                        v &= v - 1;
+                        csr_put(out, nk++, j0 + b, rs, mg.col_capacity);
+                    }
                 }
-                x[q] = v;
-                c += __popc(v);
+                for (int j = sf; j < Tb; ++j) csr_put(out, nk + (j - sf), j, rs, mg.col_capacity);
+                args.row_start[row_id] = (int32_t)rs;
+                args.row_count[row_id] = nk + (Tb - sf);
             }
-            int incl = c;
-            #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) {
-                const int a = __shfl_up_sync(hmask, incl, o, 16);
-                if (hl >= o) incl += a;
-            }
-            const int nk = __shfl_sync(hmask, incl, 15, 16);
-            int p = incl - c;
-            #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t v = x[q];
-                while (v) { const int b = __ffs(v) - 1; v &= v - 1; hstage[p++] = 32 * (4 * hl + q) + b; }
-            }
-            __syncwarp(hmask);
-            for (int p2 = hl; p2 < nk; p2 += 16) csr_put(out, p2, hstage[p2], rs, mg.col_capacity);
-            for (int j = sf + hl; j < Tb; j += 16) csr_put(out, nk + (j - sf), j, rs, mg.col_capacity);
-            if (hl == 0) { args.row_start[row_id] = (int32_t)rs; args.row_count[row_id] = nk + (Tb - sf); }
-            __syncwarp(hmask);
         }
     }
 }
