@@ -755,10 +755,11 @@ __global__ void __launch_bounds__(256) topn_overflow_kernel(const TopnArgs args)
 // query-block row: a CTA of one warp takes 32 rows of an item.  Per row:
 //   1. The bin b* of coarse >> 3 that holds the n-th largest code (suffix sums
 //      of the two row sets' histograms).
-//   2. One pass over the row's coarse and fine codes (word-major layout: the
-//      warp's loads are coalesced): coarse codes above bin b* set their bits in
-//      the row's bitmap at once; the keys of bin b* (about a dozen) are kept
-//      aside with their 16-bit code.
+//   2. One pass over the row's coarse codes (word-major layout: the warp's
+//      loads are coalesced; four groups of 32 keys in flight): coarse codes
+//      above bin b* set their bits in the row's bitmap at once; the keys of
+//      bin b* (about a dozen) are kept aside with their coarse code.  The fine
+//      bytes are read only for the keys of c* that step 3 ranks.
 //   3. From those, the coarse code c* holding the n-th largest and how many
 //      keys of c* are kept (need of m); keys of bin b* above c* are kept.  If
 //      some keys of c* are dropped (need < m): where a coarse code is narrower
@@ -788,7 +789,7 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
     const int row_end = min(mg.sink_first, Tb);
     const int sf = mg.sink_first;                          // <= Tb
     uint32_t* bm = reinterpret_cast<uint32_t*>(smem_raw);              // [32][BS]
-    uint32_t* cand = bm + 32 * BS;                                       // [BCAP][32]: code16 << 16 | j
+    uint32_t* cand = bm + 32 * BS;                                       // [BCAP][32]: coarse << 24 | j
     const int64_t units = args.BH * mtiles * 4;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
         const int64_t item = u >> 2;
@@ -824,26 +825,24 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
             const uint32_t* fw = args.fine + wbase;
             const float width = args.width[item * 128 + rl];       // loaded early: used after the pass
             int nb = 0;
-            // codes and fine bytes of groups g + 1 and g + 2 in flight while group g is read
-            uint32_t ca[8], fa[8], cb[8], fb[8];
+            // the coarse codes of groups g + 1 .. g + 4 in flight while group g is read
+            // (the fine bytes are read later, for the few keys that are ranked)
+            uint32_t ca[8], cb[8], cc[8], cd[8];
             #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 ca[k] = cw[(size_t)k * 128];
-                fa[k] = fw[(size_t)k * 128];
                 cb[k] = (G > 1) ? cw[(size_t)(8 + k) * 128] : 0u;
-                fb[k] = (G > 1) ? fw[(size_t)(8 + k) * 128] : 0u;
+                cc[k] = (G > 2) ? cw[(size_t)(16 + k) * 128] : 0u;
+                cd[k] = (G > 3) ? cw[(size_t)(24 + k) * 128] : 0u;
             }
             #pragma unroll 1
             for (int g = 0; g < G; ++g) {
-                uint32_t w[8], f[8];
+                uint32_t w[8];
                 #pragma unroll
-                for (int k = 0; k < 8; ++k) { w[k] = ca[k]; f[k] = fa[k]; ca[k] = cb[k]; fa[k] = fb[k]; }
-                if (g + 2 < G) {
+                for (int k = 0; k < 8; ++k) { w[k] = ca[k]; ca[k] = cb[k]; cb[k] = cc[k]; cc[k] = cd[k]; }
+                if (g + 4 < G) {
                     #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        cb[k] = cw[(size_t)(8 * (g + 2) + k) * 128];
-                        fb[k] = fw[(size_t)(8 * (g + 2) + k) * 128];
-                    }
+                    for (int k = 0; k < 8; ++k) cd[k] = cw[(size_t)(8 * (g + 4) + k) * 128];
                 }
                 const int nv = Tb - 32 * g;
                 const uint32_t vm = (nv >= 32) ? 0xffffffffu : ((1u << nv) - 1u);
@@ -857,10 +856,7 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
                 while (inb) {
                     const int b = __ffs(inb) - 1;
                     inb &= inb - 1;
-                    if (nb < BCAP) {
-                        const uint32_t code16 = (byte_of8(w, b) << 8) | byte_of8(f, b);
-                        cand[nb * 32 + lane] = (code16 << 16) | (uint32_t)(32 * g + b);
-                    }
+                    if (nb < BCAP) cand[nb * 32 + lane] = (byte_of8(w, b) << 24) | (uint32_t)(32 * g + b);
                     ++nb;
                 }
                 brow[g] = bits & vm;
@@ -894,20 +890,26 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
                     if (cstar == 0 || cstar == 255 || m > RCAP) {
                         rk = 2;
                     } else {
-                        // rank by (fine desc, j asc): key = fine << 16 | (0xFFFF - j)
-                        uint32_t key[RCAP];
+                        // rank by (fine desc, j asc): key = fine << 16 | (0xFFFF - j); the
+                        // fine bytes of the m keys of c* are read together (one round trip)
+                        int jr[RCAP];
                         #pragma unroll
-                        for (int y = 0; y < RCAP; ++y) key[y] = 0u;
+                        for (int y = 0; y < RCAP; ++y) jr[y] = 0;
                         int c = 0;
                         for (int e = 0; e < nb; ++e) {
                             const uint32_t x = cand[e * 32 + lane];
                             if ((x >> 24) == cstar) {
-                                const uint32_t kv = (((x >> 16) & 255u) << 16) | (0xFFFFu - (x & 0xFFFFu));
                                 #pragma unroll
-                                for (int y = 0; y < RCAP; ++y) key[y] = (y == c) ? kv : key[y];
+                                for (int y = 0; y < RCAP; ++y) jr[y] = (y == c) ? (int)(x & 0xFFFFu) : jr[y];
                                 ++c;
                             }
                         }
+                        uint32_t key[RCAP];
+                        #pragma unroll
+                        for (int y = 0; y < RCAP; ++y) key[y] = (y < m) ? fw[(size_t)(jr[y] >> 2) * 128] : 0u;
+                        #pragma unroll
+                        for (int y = 0; y < RCAP; ++y)
+                            key[y] = (y < m) ? ((((key[y] >> (8 * (jr[y] & 3))) & 255u) << 16) | (0xFFFFu - (uint32_t)jr[y])) : 0u;
                         uint32_t f_last = 0, f_next = 256;
                         #pragma unroll
                         for (int y = 0; y < RCAP; ++y) {
