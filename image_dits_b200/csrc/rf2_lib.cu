@@ -527,7 +527,7 @@ static int launch_topn(const Checked& c, const MaskGeo& mg, const MaskWs& w, int
     if (r != RF2_OK) return r;
     // rows with too many keys near their threshold for topn_rows_kernel (rare; the
     // launch returns at once when there are none)
-    topn_overflow_kernel<D><<<sms, 256, ovf_smem, s>>>(a);
+    topn_overflow_kernel<D><<<sms, 512, ovf_smem, s>>>(a);
     return launch_status();
 }
 

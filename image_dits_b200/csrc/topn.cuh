@@ -523,7 +523,7 @@ topn_codes_kernel(const __grid_constant__ CUtensorMap tm_a_hi, const __grid_cons
 // threshold code holds too many keys for topn_rows_kernel, most of them rows
 // whose sampled bracket missed the threshold (their c* is a saturated code).
 template <int D>
-__global__ void __launch_bounds__(256) topn_overflow_kernel(const TopnArgs args)
+__global__ void __launch_bounds__(512) topn_overflow_kernel(const TopnArgs args)
 {
     constexpr int E = D / 32;                              // q^ elements per lane in a dot product
     constexpr int WMAX = 16;                               // code words per lane (T_b <= 2048)
