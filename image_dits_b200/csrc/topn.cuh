@@ -770,9 +770,10 @@ __global__ void __launch_bounds__(512) topn_overflow_kernel(const TopnArgs args)
 //      64 keys in bin b*, more than 16 keys of c* to rank, more than 4 keys
 //      tied in the fine code, or its threshold in a saturated code (0 or 255:
 //      the bracket missed) is listed for topn_overflow_kernel.
-//   4. Each thread writes its own row: the kept bits of its bitmap in
-//      ascending order, then the sink columns; sink rows (and keep = 1) keep
-//      every block.  The 32 rows go out in parallel.
+//   4. Each thread writes its own row's kept keys below the sink columns (the
+//      kept bits of its bitmap in ascending order), the 32 rows in parallel;
+//      the warp then writes the sink columns of each row, and all of a sink
+//      row (or of every row at keep = 1), one row at a time, coalesced.
 template <int D>
 __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
 {
@@ -1016,35 +1017,44 @@ __global__ void __launch_bounds__(32, 12) topn_rows_kernel(const TopnArgs args)
                 args.overflow[1 + at] = (int32_t)(bh * Tb + i);
             }
         }
-        // 4. the CSR rows: thread r writes row r from its own bitmap (rows stride
-        // BS, odd: the lanes' words sit in distinct banks), kept keys below the
-        // sink columns in ascending order, then the sink columns.  The rows are
-        // written in parallel; each lane's stores run through its row in order.
-        if (rk < 2) {
-            const int64_t row_id = bh * Tb + i;
+        // 4. the CSR rows: thread r writes the kept keys below the sink columns
+        // of row r from its own bitmap (rows stride BS, odd: the lanes' words
+        // sit in distinct banks), in ascending order, the 32 rows in parallel;
+        // then the whole warp writes, one row at a time and coalesced, the
+        // sink columns of every row and all of a row that keeps every block.
+        int nk = 0;
+        if (rk == 0) {
+            const uint32_t* brow = bm + lane * BS;
             const int64_t rs = row_offset(mg, bh, i);
             int32_t* out = args.col_idx + rs;
-            if (rk == 1) {
-                for (int j = 0; j < Tb; ++j) csr_put(out, j, j, rs, mg.col_capacity);
-                args.row_start[row_id] = (int32_t)rs;
-                args.row_count[row_id] = Tb;
-            } else {
-                const uint32_t* brow = bm + lane * BS;
-                const int wl = (sf + 31) >> 5;             // bitmap words below the sink columns
-                int nk = 0;
-                for (int wi = 0; wi < wl; ++wi) {
-                    uint32_t v = brow[wi];
-                    const int j0 = 32 * wi;
-                    if (j0 + 32 > sf) v &= (1u << (sf - j0)) - 1u;
-                    while (v) {
-                        const int b = __ffs(v) - 1;
-                        v &= v - 1;
-                        csr_put(out, nk++, j0 + b, rs, mg.col_capacity);
-                    }
+            const int wl = (sf + 31) >> 5;                 // bitmap words below the sink columns
+            for (int wi = 0; wi < wl; ++wi) {
+                uint32_t v = brow[wi];
+                const int j0 = 32 * wi;
+                if (j0 + 32 > sf) v &= (1u << (sf - j0)) - 1u;
+                while (v) {
+                    const int b = __ffs(v) - 1;
+                    v &= v - 1;
+                    csr_put(out, nk++, j0 + b, rs, mg.col_capacity);
                 }
-                for (int j = sf; j < Tb; ++j) csr_put(out, nk + (j - sf), j, rs, mg.col_capacity);
+            }
+        }
+        uint32_t todo = __ballot_sync(0xffffffffu, rk < 2);
+        while (todo) {
+            const int r = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const int rkr = __shfl_sync(0xffffffffu, rk, r);
+            const int nkr = __shfl_sync(0xffffffffu, nk, r);
+            const int ir = m0 + (rl - lane) + r;
+            const int64_t row_id = bh * Tb + ir;
+            const int64_t rs = row_offset(mg, bh, ir);
+            int32_t* out = args.col_idx + rs;
+            const int j_from = (rkr == 1) ? 0 : sf;        // every block, or the sink columns
+            const int base = (rkr == 1) ? 0 : nkr;
+            for (int j = j_from + lane; j < Tb; j += 32) csr_put(out, base + (j - j_from), j, rs, mg.col_capacity);
+            if (lane == 0) {
                 args.row_start[row_id] = (int32_t)rs;
-                args.row_count[row_id] = nk + (Tb - sf);
+                args.row_count[row_id] = base + (Tb - j_from);
             }
         }
     }
