@@ -265,7 +265,9 @@ def test_long_rows_selection(keep, sink):
 
 @pytest.mark.parametrize("name,wl", _small_cases() + [("image", WORKLOADS["image"]),
                                                       ("long_rows", Workload("long", 1, 2, 128, 4, 64, 144, 2, 8, 8,
-                                                                             0.2, True, (44, 42, 42)))])
+                                                                             0.2, True, (44, 42, 42))),
+                                                      ("long_rows_keep_all", Workload("long", 1, 2, 128, 4, 64, 144, 2,
+                                                                                      8, 8, 1.0, False, (44, 42, 42)))])
 def test_mask_from_codes(name, wl, monkeypatch):
     """The selection from 16-bit score codes (the path of large calls), forced
     on small ones: the masks match the oracle outside the tie band, and the
