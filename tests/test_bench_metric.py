@@ -3,7 +3,9 @@ over the kept (query block i, key block j) pairs, r_i and c_j the valid
 tokens of the blocks (the last block of a sequence may be short), and the
 mask's algorithmic bytes are Q and K read once plus the CSR written.  Both
 are checked against a brute-force sum over random CSR masks laid out the way
-the library writes them (ascending rows with gaps between them)."""
+the library writes them (ascending rows with gaps between them).  The
+reference arm (the oracle on the host's cores) is run once on the small
+workload for its JSON line."""
 from dataclasses import replace
 from types import SimpleNamespace
 
@@ -97,3 +99,24 @@ def test_attention_traffic_figure_covers_the_compulsory_bytes():
     at d = 128: 1,024 bytes) and not far above it (K/V re-reads hit L2)."""
     assert 1024 <= bench.ATTN_DRAM_BYTES_PER_TOKEN_HEAD <= 1.2 * 1024
     assert len(bench.ATTN_TRAFFIC_BUILD) >= 7
+
+
+def test_reference_arm_line():
+    """`bench.py --impl reference` (the oracle on the host's cores, the arm the
+    driver times beside the library) runs without a GPU and prints one JSON
+    line with the contract's keys."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "TFLOP/s"
+    assert d["value"] > 0 and d["ms_per_step"] > 0 and d["higher_is_better"] is True
+    assert d["steps"] == 1 and d["warmup"] >= 3 and d["n_gpus"] == 1
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
