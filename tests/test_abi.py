@@ -264,3 +264,18 @@ def test_static_scratch_size_limit_on_host(L):
         if not fits:
             st = L.rf2_predict_mask_static(ctypes.byref(g), fake, fake, 0.2, fake, fake, fake, None)
             assert st == rf2.RF2_ERR_INSUFFICIENT_WORKSPACE
+
+
+def test_no_fallback_without_the_library_or_a_gpu_tensor(L, tmp_path):
+    """The binding has no CPU path: a missing library raises, and host tensors
+    given to a device call are refused before anything reaches the library."""
+    import torch
+    with pytest.raises(RuntimeError):
+        rf2.load(str(tmp_path / "librf2.so"))
+    g = rf2.geometry_of(WORKLOADS["tiny"])
+    wl = WORKLOADS["tiny"]
+    x = torch.zeros(wl.batch, wl.heads, wl.num_tokens, wl.head_dim, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        rf2.permute(g, x)
+    with pytest.raises(ValueError):
+        rf2.unpermute(g, x)
