@@ -37,7 +37,7 @@ def _worker(rank, world, port, out):
 def test_two_rank_combination():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:     # no fork of this (threaded) process
         out = m.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
         res = dict(out)
@@ -80,7 +80,7 @@ def test_head_split_reassembles_one_call():
     from split_case import SPLIT_WL, oracle_call
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:     # no fork of this (threaded) process
         out = m.dict()
         mp.start_processes(_split_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
         res = dict(out)
